@@ -1,0 +1,156 @@
+/*
+ * sq_w8a8.h -- C ABI of the SmoothQuant W8A8 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The method (SmoothQuant): a linear layer Y = X W is rewritten exactly as
+ * Y = (X diag(s)^-1)(diag(s) W), with a per-input-channel migration factor
+ *     s_j = max|X_j|^alpha / max|W_j|^(1 - alpha),
+ * so that activation outliers move into the weights; the smoothed weights are
+ * quantised per output channel and the smoothed activations per token to
+ * symmetric INT8, and the product runs as an INT8 x INT8 -> int32 GEMM whose
+ * epilogue multiplies back the two scales.
+ *   Pages: "4.2 W8A8 量化与 SmoothQuant" (sec. 3 equivalence, sec. 4 factor and alpha,
+ *   sec. 6 LayerNorm folding, sec. 7.1 calibration pipeline and granularity);
+ *   "量化：只压权重，与训练后量化（PTQ）", SmoothQuant section (W_j is row j of W;
+ *   per-token / per-channel scales factor out of the GEMM);
+ *   "SmoothQuant大模型平滑量化技术", Python demo (scale = max|.|/127, round, clip +-127).
+ *
+ * Conventions shared by every call
+ *   - Every pointer except `stream` and the documented host-side outputs is a DEVICE
+ *     pointer owned by the caller.  The library allocates no memory and keeps no
+ *     state besides cached device properties and a device-side error word.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
+ *     enqueues work on it and returns; nothing synchronises.
+ *   - Matrices are row-major with a leading dimension `ld*` counted in elements.
+ *     bf16 (SQ_BF16) and fp32 (SQ_F32) inputs need 16-byte aligned base pointers,
+ *     rows that are a multiple of 16 bytes (cols * elt % 16 == 0) and ld * elt % 16 == 0.
+ *   - Arithmetic: IEEE binary32, round to nearest even, one rounding per written
+ *     operation (no contraction).  int8 codes are clamp(rne(v / scale), -127, 127);
+ *     a scale of 0 (all-zero row or column) gives all-zero codes.
+ *   - Errors: arguments are validated on the host before anything is enqueued and a
+ *     bad argument returns its status with nothing launched.  A failed launch returns
+ *     SQ_ERR_CUDA.  Faults inside a kernel surface at the caller's next
+ *     synchronisation.  A kernel whose bounded internal wait runs out stops early and
+ *     records a code readable with sq_device_error().
+ *   - Sizes: a zero-sized problem returns SQ_OK and launches nothing, except that an
+ *     empty calibration reduction (no rows) with accumulate = 0 zero-fills `out`; calls
+ *     that need K > 0 (LayerNorm, GEMM) reject K == 0 as SQ_ERR_INVALID_ARG.
+ */
+#ifndef SQ_W8A8_H
+#define SQ_W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, ld < cols, ...      */
+  SQ_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement (K limits)    */
+  SQ_ERR_ALIGNMENT = 3,   /* pointer / row / leading dimension not 16-byte aligned      */
+  SQ_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed                      */
+  SQ_ERR_WORKSPACE = 5    /* the GEMM workspace is missing or too small                  */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_BF16 = 1, SQ_I32 = 2 } sq_dtype;
+
+/* Largest K the int32 accumulator holds: K * 127^2 <= 2^31 - 1 up to K = 133144;
+ * rounded down to a multiple of 16. */
+#define SQ_MAX_K 133136
+/* Largest K of the LayerNorm / per-token quantiser (row kept on chip). */
+#define SQ_MAX_K_ROW 65536
+
+/* sq_calib_absmax -- calibration statistics, one pass over x.
+ *   axis 0: out[j] = max_i |x[i, j]|, j < cols  (per input channel over calibration
+ *           tokens: "4.2 W8A8…" sec. 7.1 step 2, "量化…PTQ" SmoothQuant section)
+ *   axis 1: out[i] = max_j |x[i, j]|, i < rows  (per row; for weights W[K, N] row j is
+ *           input channel j: "量化…PTQ" SmoothQuant section)
+ *   x: [rows, cols] bf16 or fp32, leading dimension ld (elements).  out: fp32 [cols] or
+ *   [rows].  accumulate = 0 overwrites out; 1 takes the running max with its contents
+ *   (statistics over several calibration batches).  The result is exact (a max). */
+sq_status sq_calib_absmax(const void* x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                          int axis, int accumulate, float* out, void* stream);
+
+/* sq_calib_ln_absmax -- per-channel absmax of a LayerNorm output, without writing it:
+ *   out[j] = max_i |LN(x_i)_j|, LN(x)_j = fma((x_j - mu) * rstd, gamma_j, beta_j),
+ *   rstd = 1 / sqrt(var + eps) (biased variance, two passes, fixed reduction order of
+ *   sq_ln_smooth_quant).  This is the statistic of the linear's input when a LayerNorm
+ *   precedes it ("4.2 W8A8…" sec. 6 and 7.1).  x: [rows, K] bf16/fp32, ldx; gamma [K]
+ *   fp32; beta [K] fp32 or NULL (= 0).  K % 16 == 0, K <= SQ_MAX_K_ROW.
+ *   accumulate as for sq_calib_absmax. */
+sq_status sq_calib_ln_absmax(const void* x, sq_dtype dt, int64_t rows, int64_t K, int64_t ldx,
+                             const float* gamma, const float* beta, float eps, int accumulate,
+                             float* out, void* stream);
+
+/* sq_smooth_factors -- s_j = ax_j^alpha / aw_j^(1 - alpha) ("4.2 W8A8…" sec. 4).
+ *   ax, aw, s: fp32 [K].  0 <= alpha <= 1.  Evaluated in binary64 and rounded once to
+ *   binary32: sqrt(ax/aw) at alpha = 0.5, ax at 1, 1/aw at 0, exp(alpha log ax -
+ *   (1 - alpha) log aw) otherwise.  A channel with ax_j = 0 or aw_j = 0 gets s_j = 1. */
+sq_status sq_smooth_factors(const float* ax, const float* aw, int64_t K, float alpha, float* s,
+                            void* stream);
+
+/* sq_fold_quant_weights -- fold diag(s) into W and quantise per output channel
+ * ("4.2 W8A8…" sec. 6 and 7.1):
+ *   W'[j, k] = s_j * W[j, k]; sw[k] = max_j |W'[j, k]| / 127;
+ *   Wq[k, j] = clamp(rne(W'[j, k] / sw[k]), -127, 127)
+ *   gamma_f[j] = gamma[j] / s_j and beta_f[j] = beta[j] / s_j (LayerNorm folding),
+ *   each written only when both its input and output pointers are non-NULL.
+ *   W: [K, N] bf16/fp32 (row j = input channel), leading dimension ldw.
+ *   Wq: int8 [N, K], K contiguous (the GEMM's K-major B operand), 16-byte aligned.
+ *   sw: fp32 [N].  K % 16 == 0, K <= SQ_MAX_K. */
+sq_status sq_fold_quant_weights(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                                const float* s, const float* gamma, const float* beta,
+                                int8_t* Wq, float* sw, float* gamma_f, float* beta_f,
+                                void* stream);
+
+/* sq_ln_smooth_quant -- fused LayerNorm -> X diag(s)^-1 -> per-token INT8
+ * ("4.2 W8A8…" sec. 6 and 7.1; "量化…PTQ" per-token activations):
+ *   LayerNorm mode (gamma_f != NULL, s == NULL): y = LN(x) with the folded gamma' = gamma/s,
+ *     beta' = beta/s (beta_f may be NULL = 0); statistics as in sq_calib_ln_absmax.
+ *   plain mode (gamma_f == NULL, s != NULL): y_j = x_j / s_j (input from a previous GEMM).
+ *   sx[m] = max_j |y[m, j]| / 127;  xq[m, j] = clamp(rne(y[m, j] / sx[m]), -127, 127).
+ *   x: [M, K] bf16/fp32, ldx.  xq: int8 [M, K] dense, 16-byte aligned.  sx: fp32 [M].
+ *   K % 16 == 0, K <= SQ_MAX_K_ROW.  Exactly one of gamma_f and s is non-NULL. */
+sq_status sq_ln_smooth_quant(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                             const float* gamma_f, const float* beta_f, const float* s, float eps,
+                             int8_t* xq, float* sx, void* stream);
+
+/* sq_w8a8_gemm -- INT8 x INT8 -> int32 GEMM on the tcgen05 tensor cores with the dequant
+ * epilogue ("4.2 W8A8…" intro: the GEMM runs on INT8 tensor cores; "量化…PTQ": per-token
+ * and per-channel scales are multiplied back after the GEMM):
+ *   acc[m, n] = sum_j xq[m, j] * wq[n, j]   (exact int32)
+ *   ydt = SQ_BF16: y[m, n] = bf16_rne(((float)acc[m, n] * sx[m]) * sw[n])
+ *   ydt = SQ_F32:  y[m, n] = ((float)acc[m, n] * sx[m]) * sw[n]
+ *   ydt = SQ_I32:  y[m, n] = acc[m, n]            (sx, sw may then be NULL)
+ *   xq: int8 [M, K] dense; wq: int8 [N, K] dense; both 16-byte aligned; K % 16 == 0,
+ *   K <= SQ_MAX_K.  y: [M, N] with leading dimension ldy >= N, aligned to its element
+ *   size (16-byte aligned rows take the vectorised store path).  M == 0 or N == 0 is a
+ *   no-op; K == 0 is invalid.
+ *   workspace: device scratch of at least sq_w8a8_gemm_workspace_size(M, N, K) bytes
+ *   (may be NULL when that size is 0), 256-byte aligned; its contents on entry do not
+ *   matter.  Calls that share a workspace must be ordered on one stream. */
+sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                       int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes sq_w8a8_gemm needs for this shape on the current device (0 when the
+ * launch it picks does not split K).  Returns (size_t)-1 for invalid sizes. */
+size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* Reads (and with clear != 0 resets) the device-side error word of the current device:
+ * 0 when no kernel gave up on a bounded wait.  Synchronises `stream`. */
+sq_status sq_device_error(unsigned int* code, int clear, void* stream);
+
+/* Human-readable name of a status. */
+const char* sq_status_string(sq_status status);
+
+/* ABI version of this header (major * 100 + minor). */
+int sq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_W8A8_H */

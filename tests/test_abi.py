@@ -1,0 +1,156 @@
+"""The C-ABI library builds for sm_100a, loads, exports every symbol its header declares,
+and validates arguments on the host before touching the device.  CPU only: every call
+below returns its status before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w8a8_smoothquant_gemm_b200 as sq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sq_w8a8.h")
+
+INVALID, UNSUPPORTED, ALIGN, WORKSPACE = 1, 2, 3, 5
+F32, BF16, I32 = 0, 1, 2
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported():
+    L = sq.lib()
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_library_has_no_cuda_runtime_or_driver_link_dependency():
+    # the runtime is linked statically and the driver is reached through the runtime's
+    # entry-point query, so the library loads on a machine without a GPU driver
+    import subprocess
+    out = subprocess.run(["ldd", sq.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcudart" not in out and "libcuda.so" not in out
+
+
+def test_status_strings_and_version():
+    L = sq.lib()
+    assert L.sq_status_string(0) == b"SQ_OK"
+    assert L.sq_status_string(5) == b"SQ_ERR_WORKSPACE"
+    assert L.sq_abi_version() == 100
+
+
+# fake, never dereferenced device addresses with chosen alignment
+A16 = ctypes.c_void_p(0x10000)
+A16b = ctypes.c_void_p(0x20000)
+A16c = ctypes.c_void_p(0x30000)
+A8 = ctypes.c_void_p(0x10008)
+NULL = None
+
+
+def test_calib_absmax_validation():
+    f = sq.lib().sq_calib_absmax
+    assert f(A16, BF16, 4, 64, 64, 2, 0, A16b, NULL) == INVALID        # bad axis
+    assert f(A16, BF16, 4, 64, 64, 0, 3, A16b, NULL) == INVALID        # bad accumulate
+    assert f(A16, I32, 4, 64, 64, 0, 0, A16b, NULL) == INVALID         # int32 input
+    assert f(NULL, BF16, 4, 64, 64, 0, 0, A16b, NULL) == INVALID       # null x
+    assert f(A16, BF16, 4, 64, 32, 0, 0, A16b, NULL) == INVALID        # ld < cols
+    assert f(A16, BF16, -1, 64, 64, 0, 0, A16b, NULL) == INVALID       # negative rows
+    assert f(A8, BF16, 4, 64, 64, 0, 0, A16b, NULL) == ALIGN           # misaligned x
+    assert f(A16, BF16, 4, 60, 64, 0, 0, A16b, NULL) == ALIGN          # 120-byte rows
+    assert f(A16, F32, 4, 64, 66, 0, 0, A16b, NULL) == ALIGN           # ld not 16 bytes
+    assert f(A16, BF16, 4, 64, 64, 0, 0, NULL, NULL) == INVALID        # null out
+    assert f(A16, BF16, 4, 0, 0, 0, 0, NULL, NULL) == 0                # nothing to do
+
+
+def test_calib_ln_absmax_validation():
+    f = sq.lib().sq_calib_ln_absmax
+    assert f(A16, BF16, 4, 64, 64, NULL, NULL, 1e-5, 0, A16b, NULL) == INVALID     # null gamma
+    assert f(A16, BF16, 4, 0, 0, A16c, NULL, 1e-5, 0, A16b, NULL) == INVALID       # K = 0
+    assert f(A16, BF16, 4, 24, 24, A16c, NULL, 1e-5, 0, A16b, NULL) == ALIGN       # 48-byte rows, K % 16
+    assert f(A16, BF16, 4, 65552, 65552, A16c, NULL, 1e-5, 0, A16b, NULL) == UNSUPPORTED
+    assert f(A16, F32, 4, 32784, 32784, A16c, NULL, 1e-5, 0, A16b, NULL) == UNSUPPORTED
+    assert f(A16, BF16, 4, 64, 64, A16c, NULL, -1.0, 0, A16b, NULL) == INVALID     # eps < 0
+
+
+def test_smooth_factors_validation():
+    f = sq.lib().sq_smooth_factors
+    assert f(A16, A16b, 64, ctypes.c_float(1.5), A16c, NULL) == INVALID
+    assert f(A16, A16b, 64, ctypes.c_float(-0.1), A16c, NULL) == INVALID
+    assert f(A16, A16b, 64, ctypes.c_float(float("nan")), A16c, NULL) == INVALID
+    assert f(NULL, A16b, 64, ctypes.c_float(0.5), A16c, NULL) == INVALID
+    assert f(A16, A16b, -3, ctypes.c_float(0.5), A16c, NULL) == INVALID
+    assert f(NULL, NULL, 0, ctypes.c_float(0.5), NULL, NULL) == 0
+
+
+def test_fold_validation():
+    f = sq.lib().sq_fold_quant_weights
+    ok = dict(W=A16, dt=BF16, K=64, N=32, ldw=32, s=A16b, g=NULL, b=NULL, wq=A16c, sw=A16b, gf=NULL, bf=NULL)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return f(a["W"], a["dt"], a["K"], a["N"], a["ldw"], a["s"], a["g"], a["b"], a["wq"], a["sw"], a["gf"],
+                 a["bf"], NULL)
+
+    assert call(s=NULL) == INVALID
+    assert call(wq=NULL) == INVALID
+    assert call(K=40, ldw=32) == ALIGN                     # K % 16 != 0
+    assert call(wq=A8) == ALIGN
+    assert call(N=36, ldw=36) == ALIGN                     # 72-byte rows
+    assert call(K=0) == 0 and call(N=0, ldw=0) == 0
+
+
+SQ_MAX_K_PLUS = 133152  # next multiple of 16 above the int32 accumulator bound
+
+
+def test_fold_rejects_k_beyond_int32_range():
+    f = sq.lib().sq_fold_quant_weights
+    assert f(A16, BF16, SQ_MAX_K_PLUS, 32, 32, A16b, NULL, NULL, A16c, A16b, NULL, NULL, NULL) == UNSUPPORTED
+
+
+def test_ln_smooth_quant_validation():
+    f = sq.lib().sq_ln_smooth_quant
+    # both modes / neither mode
+    assert f(A16, BF16, 4, 64, 64, A16b, NULL, A16c, 1e-5, A16c, A16b, NULL) == INVALID
+    assert f(A16, BF16, 4, 64, 64, NULL, NULL, NULL, 1e-5, A16c, A16b, NULL) == INVALID
+    assert f(A16, BF16, 4, 64, 64, NULL, A16b, A16c, 1e-5, A16c, A16b, NULL) == INVALID   # beta without gamma
+    assert f(A16, BF16, 4, 64, 64, A8, NULL, NULL, 1e-5, A16c, A16b, NULL) == ALIGN
+    assert f(A16, BF16, 4, 40, 40, NULL, NULL, A16c, 1e-5, A16c, A16b, NULL) == ALIGN      # K % 16
+    assert f(A16, BF16, 4, 64, 64, NULL, NULL, A16c, 1e-5, NULL, A16b, NULL) == INVALID    # null xq
+    assert f(A16, BF16, 4, 65552, 65552, NULL, NULL, A16c, 1e-5, A16c, A16b, NULL) == UNSUPPORTED
+    assert f(A16, BF16, 0, 64, 64, NULL, NULL, A16c, 1e-5, NULL, NULL, NULL) == 0          # M = 0
+
+
+def test_gemm_validation():
+    f = sq.lib().sq_w8a8_gemm
+
+    def call(xq=A16, sx=A16b, wq=A16c, sw=A16b, M=8, N=32, K=64, y=A16, ydt=BF16, ldy=32, ws=NULL, wsb=0):
+        return f(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, wsb, NULL)
+
+    assert call(K=0) == INVALID
+    assert call(ydt=7) == INVALID
+    assert call(ldy=16) == INVALID
+    assert call(xq=NULL) == INVALID
+    assert call(sx=NULL) == INVALID                 # scales needed for bf16 output
+    assert call(K=40) == ALIGN
+    assert call(wq=A8) == ALIGN
+    assert call(y=ctypes.c_void_p(0x10001)) == ALIGN  # output not aligned to its element
+    assert call(ws=ctypes.c_void_p(0x10010)) == ALIGN
+    assert call(K=SQ_MAX_K_PLUS) == UNSUPPORTED
+    assert call(M=0) == 0 and call(N=0, ldy=0) == 0
+
+
+def test_workspace_size_validation():
+    f = sq.lib().sq_w8a8_gemm_workspace_size
+    assert f(4, 4, 0) == ctypes.c_size_t(-1).value
+    assert f(4, 4, 24) == ctypes.c_size_t(-1).value
+    assert f(0, 64, 64) == 0
+
+
+def test_device_error_null_pointer():
+    assert sq.lib().sq_device_error(NULL, 0, NULL) == INVALID

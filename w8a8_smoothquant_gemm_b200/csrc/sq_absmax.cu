@@ -1,0 +1,240 @@
+// sq_absmax.cu -- calibration statistics of SmoothQuant ("4.2 W8A8 量化与 SmoothQuant",
+// sec. 4 and 7.1; "量化：只压权重，与训练后量化（PTQ）", SmoothQuant section):
+//   per-input-channel activation absmax  max_i |X_ij|      (column max, axis 0)
+//   per-input-channel weight absmax       max_k |W_jk|      (row max of W[K, N], axis 1)
+//   per-channel absmax of a LayerNorm output, computed without writing it.
+//
+// All three are HBM-bound single passes: 16-byte vector loads that bypass L1, a
+// per-thread running max, a block reduction, and one atomicMax per column per block on
+// the float bit pattern (monotone for non-negative floats, so the result is exact and
+// independent of order).
+#include "sq_rowln.cuh"
+
+namespace sqk {
+
+// ---------------------------------------------------------------------------- axis 0
+// Block = 32 column vectors (x) x 8 row lanes (y).  A warp reads 32 consecutive
+// 16-byte vectors of one row (512 contiguous bytes).  Each thread walks rows
+// r = blockIdx.y * 8 + threadIdx.y + k * gridDim.y * 8, four loads in flight.
+constexpr int COL_VX = 32, COL_RY = 8, COL_UNROLL = 4;
+
+template <bool BF16>
+__global__ void __launch_bounds__(COL_VX * COL_RY)
+absmax_cols_kernel(const char* __restrict__ x, int64_t rows, int64_t nvec, int64_t ld_bytes,
+                   float* __restrict__ out) {
+  constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
+  __shared__ float red[COL_RY][COL_VX * EPV + 1];
+  const int64_t vec = (int64_t)blockIdx.x * COL_VX + threadIdx.x;
+  float m[EPV];
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) m[e] = 0.0f;
+  if (vec < nvec) {
+    const int64_t rstep = (int64_t)gridDim.y * COL_RY;
+    int64_t r = (int64_t)blockIdx.y * COL_RY + threadIdx.y;
+    const char* p = x + vec * 16;
+    for (; r + (COL_UNROLL - 1) * rstep < rows; r += COL_UNROLL * rstep) {
+      uint4 v[COL_UNROLL];
+#pragma unroll
+      for (int u = 0; u < COL_UNROLL; ++u) v[u] = ldg_stream16(p + (r + u * rstep) * ld_bytes);
+#pragma unroll
+      for (int u = 0; u < COL_UNROLL; ++u) {
+        if (BF16) {
+          float f[8];
+          unpack8_bf16(v[u], f);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+        } else {
+          const float f[4] = {__uint_as_float(v[u].x), __uint_as_float(v[u].y), __uint_as_float(v[u].z),
+                              __uint_as_float(v[u].w)};
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+        }
+      }
+    }
+    for (; r < rows; r += rstep) {
+      const uint4 v = ldg_stream16(p + r * ld_bytes);
+      if (BF16) {
+        float f[8];
+        unpack8_bf16(v, f);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+      } else {
+        const float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w)};
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) red[threadIdx.y][threadIdx.x * EPV + e] = m[e];
+  __syncthreads();
+  // 256 threads finish the COL_VX * EPV columns of this block.
+  const int tid = threadIdx.y * COL_VX + threadIdx.x;
+  for (int c = tid; c < COL_VX * EPV; c += COL_VX * COL_RY) {
+    float v = red[0][c];
+#pragma unroll
+    for (int y = 1; y < COL_RY; ++y) v = fmaxf(v, red[y][c]);
+    const int64_t col = (int64_t)blockIdx.x * COL_VX * EPV + c;
+    if (col < nvec * EPV) atomic_max_nonneg(out + col, v);
+  }
+}
+
+// ---------------------------------------------------------------------------- axis 1
+// One block of 256 threads per row; the row is read as 16-byte vectors.
+template <bool BF16>
+__global__ void __launch_bounds__(256)
+absmax_rows_kernel(const char* __restrict__ x, int64_t rows, int64_t nvec, int64_t ld_bytes,
+                   int accumulate, float* __restrict__ out) {
+  __shared__ float red[ROW_WARPS + 1];
+  const int64_t r = blockIdx.x;
+  const char* p = x + r * ld_bytes;
+  float m = 0.0f;
+  int64_t v = threadIdx.x;
+  for (; v + 3 * 256 < nvec; v += 4 * 256) {
+    uint4 q[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) q[u] = ldg_stream16(p + (v + u * 256) * 16);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (BF16) {
+        float f[8];
+        unpack8_bf16(q[u], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+      } else {
+        m = fmaxf(fmaxf(m, fabsf(__uint_as_float(q[u].x))), fabsf(__uint_as_float(q[u].y)));
+        m = fmaxf(fmaxf(m, fabsf(__uint_as_float(q[u].z))), fabsf(__uint_as_float(q[u].w)));
+      }
+    }
+  }
+  for (; v < nvec; v += 256) {
+    const uint4 q = ldg_stream16(p + v * 16);
+    if (BF16) {
+      float f[8];
+      unpack8_bf16(q, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    } else {
+      m = fmaxf(fmaxf(m, fabsf(__uint_as_float(q.x))), fabsf(__uint_as_float(q.y)));
+      m = fmaxf(fmaxf(m, fabsf(__uint_as_float(q.z))), fabsf(__uint_as_float(q.w)));
+    }
+  }
+  m = block_max(m, red);
+  if (threadIdx.x == 0) out[r] = accumulate ? fmaxf(out[r], m) : m;
+}
+
+// ---------------------------------------------------------------------------- LayerNorm output
+// Blocks loop over rows; each thread keeps the running max of the elements of its own
+// chunks in shared memory (no conflicts), then one atomicMax per column per block.
+// With rows_atomic set (K too large for shared memory) the running max goes straight
+// to global memory with an atomic per element per row.
+template <bool BF16, int MAXC>
+__global__ void __launch_bounds__(ROW_THREADS)
+calib_ln_absmax_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t ld_bytes,
+                       const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                       int rows_atomic, float* __restrict__ out) {
+  extern __shared__ float colmax[];
+  __shared__ float red[2 * (ROW_WARPS + 1)];
+  const int nchunks = K / 8;
+  if (!rows_atomic)
+    for (int j = threadIdx.x; j < K; j += ROW_THREADS) colmax[j] = 0.0f;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    RowChunks<BF16, MAXC> rc;
+    rc.load(x + r * ld_bytes, nchunks);
+    float mu, rstd;
+    row_stats(rc, nchunks, K, eps, red, mu, rstd);
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+      const int c = threadIdx.x + i * ROW_THREADS;
+      if (c < nchunks) {
+        float f[8], y[8];
+        rc.get(i, f);
+        ln_chunk(f, mu, rstd, gamma, beta, c, y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (rows_atomic) atomic_max_nonneg(out + c * 8 + e, fabsf(y[e]));
+          else colmax[c * 8 + e] = fmaxf(colmax[c * 8 + e], fabsf(y[e]));
+        }
+      }
+    }
+  }
+  if (!rows_atomic) {
+    __syncthreads();
+    for (int j = threadIdx.x; j < K; j += ROW_THREADS) atomic_max_nonneg(out + j, colmax[j]);
+  }
+}
+
+}  // namespace sqk
+
+// ---------------------------------------------------------------------------- launchers
+namespace sqh {
+
+cudaError_t launch_absmax(const void* x, bool bf16, int64_t rows, int64_t cols, int64_t ld, int axis,
+                          int accumulate, float* out, cudaStream_t st) {
+  const int elt = bf16 ? 2 : 4;
+  const int64_t nvec = cols * elt / 16;
+  const int64_t ld_bytes = ld * elt;
+  if (axis == 0) {
+    if (!accumulate) {
+      cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)cols, st);
+      if (e != cudaSuccess) return e;
+    }
+    const int64_t gx = (nvec + sqk::COL_VX - 1) / sqk::COL_VX;
+    const int64_t want = (int64_t)num_sms() * 8;  // 8 blocks of 256 threads per SM
+    int64_t gy = std::max<int64_t>(1, want / gx);
+    gy = std::min<int64_t>(gy, (rows + sqk::COL_RY - 1) / sqk::COL_RY);
+    gy = std::min<int64_t>(gy, 65535);
+    dim3 grid((unsigned)gx, (unsigned)gy), block(sqk::COL_VX, sqk::COL_RY);
+    if (bf16)
+      sqk::absmax_cols_kernel<true><<<grid, block, 0, st>>>((const char*)x, rows, nvec, ld_bytes, out);
+    else
+      sqk::absmax_cols_kernel<false><<<grid, block, 0, st>>>((const char*)x, rows, nvec, ld_bytes, out);
+  } else {
+    if (bf16)
+      sqk::absmax_rows_kernel<true><<<(unsigned)rows, 256, 0, st>>>((const char*)x, rows, nvec, ld_bytes, accumulate, out);
+    else
+      sqk::absmax_rows_kernel<false><<<(unsigned)rows, 256, 0, st>>>((const char*)x, rows, nvec, ld_bytes, accumulate, out);
+  }
+  return cudaGetLastError();
+}
+
+template <bool BF16, int MAXC>
+static cudaError_t launch_calib_ln_t(const void* x, int64_t rows, int K, int64_t ld_bytes, const float* gamma,
+                                     const float* beta, float eps, float* out, cudaStream_t st) {
+  const size_t smem_cols = sizeof(float) * (size_t)K;
+  const bool rows_atomic = smem_cols > 160 * 1024;
+  const size_t smem = rows_atomic ? 0 : smem_cols;
+  auto kern = sqk::calib_ln_absmax_kernel<BF16, MAXC>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  int per_sm = 1;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sqk::ROW_THREADS, smem);
+  if (e != cudaSuccess) return e;
+  int64_t grid = std::min<int64_t>(rows, (int64_t)num_sms() * std::max(per_sm, 1));
+  kern<<<(unsigned)grid, sqk::ROW_THREADS, smem, st>>>((const char*)x, rows, K, ld_bytes, gamma, beta, eps,
+                                                       rows_atomic ? 1 : 0, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_calib_ln_absmax(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ld,
+                                   const float* gamma, const float* beta, float eps, int accumulate,
+                                   float* out, cudaStream_t st) {
+  if (!accumulate) {
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)K, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t ldb = ld * (bf16 ? 2 : 4);
+  const int need = (int)((K / 8 + sqk::ROW_THREADS - 1) / sqk::ROW_THREADS);
+  const int k = (int)K;
+#define SQ_LN_CASE(C)                                                                                   \
+  if (need <= C)                                                                                        \
+    return bf16 ? launch_calib_ln_t<true, C>(x, rows, k, ldb, gamma, beta, eps, out, st)                \
+                : launch_calib_ln_t<false, (C > 16 ? 16 : C)>(x, rows, k, ldb, gamma, beta, eps, out, st);
+  SQ_LN_CASE(1) SQ_LN_CASE(2) SQ_LN_CASE(4) SQ_LN_CASE(8) SQ_LN_CASE(16) SQ_LN_CASE(24) SQ_LN_CASE(32)
+#undef SQ_LN_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sqh

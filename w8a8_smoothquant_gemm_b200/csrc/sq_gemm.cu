@@ -1,0 +1,598 @@
+// sq_gemm.cu -- INT8 x INT8 -> int32 GEMM with the SmoothQuant dequant epilogue on the
+// 5th-generation (tcgen05) tensor cores of sm_100a.
+//
+//   acc[m, n] = sum_j xq[m, j] * wq[n, j]            exact int32
+//   y[m, n]   = bf16_rne(((float)acc * sx[m]) * sw[n])
+//
+// "4.2 W8A8 量化与 SmoothQuant" (intro, sec. 6): W8A8 lets the whole GEMM run on the INT8
+// tensor cores and the runtime kernel is a plain INT8 GEMM; "量化：只压权重，与训练后量化
+// （PTQ）", SmoothQuant section: per-token activation scales and per-output-channel weight
+// scales are constant along the summed index, so they are applied after the GEMM.
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   warp 0      one lane issues TMA loads (128-byte swizzle, no multicast) of a 128-row
+//               A tile and a BN-row B tile, 128 bytes of K each, into a STAGES-deep
+//               shared-memory ring guarded by full/empty mbarriers;
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma.cta_group::1.kind::i8
+//               (M = 128, N = BN, K = 32 per instruction) into one of two TMEM
+//               accumulators, and tcgen05.commit frees ring slots / signals the epilogue;
+//   warps 2-5   epilogue: tcgen05.ld of the int32 accumulator (warp w reads TMEM lanes
+//               32*(w%4) .. +31), scale, convert, store; the second accumulator lets the
+//               next tile's MMAs run meanwhile.
+// Operands are K-major: A = xq [M, K], B = wq [N, K].  For decode-sized M (<= 128) the
+// roles swap (A = wq, B = xq) so the weights fill the 128-row MMA dimension and the
+// tokens the N dimension; when there are fewer tiles than SMs, K is split and int32
+// partials are summed (exactly, in a fixed order) by a second kernel that also applies
+// the epilogue.  Every mbarrier wait is bounded: on expiry the kernel records a code in
+// a device error word and leaves.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "sq_common.cuh"
+
+namespace sqk {
+
+__device__ unsigned int g_error_word = 0;
+
+constexpr int BM = 128;          // MMA M: rows of the A operand per tile
+constexpr int BK = 128;          // K bytes per ring stage (one 128-byte swizzle row)
+constexpr int UMMA_K = 32;       // K per tcgen05.mma kind::i8
+constexpr int GEMM_THREADS = 192;
+constexpr unsigned long long WAIT_NS = 10ull * 1000 * 1000 * 1000;  // 10 s per wait
+
+struct GemmParams {
+  int tiles_a, tiles_b;      // tiles along A rows (BM) and B rows (BN)
+  int num_kb;                // ceil(K / BK)
+  int kb_per_split, splits;
+  int num_units;             // tiles_a * tiles_b * splits
+  int group_a;               // raster: this many A tiles share a sweep over B tiles
+  int M, N;                  // output is y[M, N]
+  const float* sx;
+  const float* sw;
+  void* y;
+  int64_t ldy;
+  int ydt;                   // SQ_BF16, SQ_F32 or SQ_I32
+  int vec_store;             // y and every output row start on a 16-byte boundary
+  int32_t* ws;               // [splits][M][N] int32 partials when splits > 1
+};
+
+// ----------------------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for the phase with the given parity to complete; false after `limit_ns`.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          unsigned long long limit_ns = WAIT_NS) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023u) == 0 && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, int8 -> int32.
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with 128-byte
+// swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (stride byte
+// offset), leading byte offset unused for swizzled K-major layouts, descriptor version 1
+// (sm_100), layout code 2 = 128-byte swizzle.  The tile base is 1024-byte aligned; the
+// k-th 32-byte step inside a row advances the start address by 32 bytes.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::i8: D = s32 (bits 4-5 = 2), A and B
+// signed 8-bit (bits 7-9, 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// 32 lanes x NCOL consecutive 32-bit TMEM columns -> NCOL registers per thread.
+template <int NCOL>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t* r);
+
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Output value of one accumulator: ((float)acc * sx) * sw, each product rounded.
+__device__ __forceinline__ float dequant(int32_t acc, float sxm, float swn) {
+  return __fmul_rn(__fmul_rn(__int2float_rn(acc), sxm), swn);
+}
+
+__device__ __forceinline__ void store_out(const GemmParams& p, int64_t m, int64_t n, int32_t acc, float sxm,
+                                          float swn) {
+  const int64_t off = m * p.ldy + n;
+  if (p.ydt == SQ_BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(dequant(acc, sxm, swn));
+  else if (p.ydt == SQ_F32) reinterpret_cast<float*>(p.y)[off] = dequant(acc, sxm, swn);
+  else reinterpret_cast<int32_t*>(p.y)[off] = acc;
+}
+
+// Unit u -> (A tile, B tile, K split).  Splits of one tile are adjacent so they run
+// concurrently; tiles are rastered in groups of group_a A tiles for L2 reuse.
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta, int& tb, int& split) {
+  split = u % p.splits;
+  const int tile = u / p.splits;
+  const int group_size = p.group_a * p.tiles_b;
+  const int group = tile / group_size;
+  const int first_a = group * p.group_a;
+  const int ga = min(p.tiles_a - first_a, p.group_a);
+  const int in_group = tile % group_size;
+  ta = first_a + in_group % ga;
+  tb = in_group / ga;
+}
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 4;
+  static constexpr int TOTAL = 1024 /* alignment slack */ + BAR_OFFSET + NUM_BARS * 8 + 16;
+  static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;  // power of two for BN in {16..256}
+};
+
+template <int BN, int STAGES, bool SWAP>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 const GemmParams p) {
+  using L = GemmSmem<BN, STAGES>;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M = 128 needs N % 16 == 0, 16..256");
+  constexpr uint32_t IDESC = idesc_i8(BM, BN);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::BAR_OFFSET;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::BAR_OFFSET + L::NUM_BARS * 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"((uint32_t)L::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t issued = 0;  // bit s: stage s has been loaded; its last load used parity bit s of `par`
+      uint32_t par = 0;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        int ta, tb, split;
+        decode_unit(p, u, ta, tb, split);
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
+            atomicOr(&g_error_word, ERR_GEMM_PRODUCER_WAIT);
+            ok = false;
+            break;
+          }
+          issued |= 1u << stage;
+          par = (par & ~(1u << stage)) | (phase << stage);
+          mbar_arrive_expect_tx(full_bar(stage), (uint32_t)L::STAGE_BYTES);
+          const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          tma_load_2d(sa, &map_a, full_bar(stage), kb * BK, ta * BM);
+          tma_load_2d(sa + L::A_BYTES, &map_b, full_bar(stage), kb * BK, tb * BN);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let the loads this thread issued land before the block exits (bounded, 100 ms)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) (void)mbar_wait(full_bar(s), (par >> s) & 1u, 100ull * 1000 * 1000);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++it) {
+        int ta, tb, split;
+        decode_unit(p, u, ta, tb, split);
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+        const int acc = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(tempty_bar(acc), aph ^ 1u)) {
+          atomicOr(&g_error_word, ERR_GEMM_MMA_WAIT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase)) {
+            atomicOr(&g_error_word, ERR_GEMM_MMA_WAIT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            tc_mma_i8(d_tmem, sw128_desc(sa + k * UMMA_K), sw128_desc(sb + k * UMMA_K), IDESC,
+                      (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        tc_commit(tfull_bar(acc));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;          // row of the A tile = TMEM lane
+    int it = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++it) {
+      int ta, tb, split;
+      decode_unit(p, u, ta, tb, split);
+      const int acc = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(tfull_bar(acc), aph)) {
+        atomicOr(&g_error_word, ERR_GEMM_EPILOGUE_WAIT);
+        break;
+      }
+      __syncwarp();  // tcgen05.ld below is .sync.aligned: reconverge after the wait loop
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int64_t arow = (int64_t)ta * BM + row;
+      constexpr int CH = BN >= 32 ? 32 : 16;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += CH) {
+        uint32_t r[CH];
+        tmem_ld<CH>(taddr + (uint32_t)c0, r);
+        tmem_wait_ld();
+        if (!SWAP) {
+          // A row = output row m; TMEM columns = output columns n
+          const int64_t m = arow;
+          const int64_t n0 = (int64_t)tb * BN + c0;
+          if (m < p.M && n0 < p.N) {
+            if (p.splits > 1) {
+              int32_t* dst = p.ws + ((int64_t)split * p.M + m) * p.N + n0;
+              for (int i = 0; i < CH; ++i)
+                if (n0 + i < p.N) dst[i] = (int32_t)r[i];
+            } else {
+              const float sxm = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m);
+              const bool full = n0 + CH <= p.N && p.vec_store;
+              if (full && p.ydt == SQ_BF16) {
+                uint32_t packed[CH / 2];
+#pragma unroll
+                for (int i = 0; i < CH; i += 2) {
+                  const float v0 = dequant((int32_t)r[i], sxm, __ldg(p.sw + n0 + i));
+                  const float v1 = dequant((int32_t)r[i + 1], sxm, __ldg(p.sw + n0 + i + 1));
+                  __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(v0), __float2bfloat16_rn(v1));
+                  packed[i / 2] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y) + m * p.ldy + n0);
+#pragma unroll
+                for (int v = 0; v < CH / 8; ++v)
+                  dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+              } else {
+                for (int i = 0; i < CH; ++i) {
+                  const int64_t n = n0 + i;
+                  if (n < p.N) store_out(p, m, n, (int32_t)r[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n));
+                }
+              }
+            }
+          }
+        } else {
+          // A row = output column n; TMEM columns = output rows m
+          const int64_t n = arow;
+          const int64_t m0 = (int64_t)tb * BN + c0;
+          if (n < p.N) {
+            if (p.splits > 1) {
+              for (int i = 0; i < CH; ++i) {
+                const int64_t m = m0 + i;
+                if (m < p.M) p.ws[((int64_t)split * p.M + m) * p.N + n] = (int32_t)r[i];
+              }
+            } else {
+              const float swn = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n);
+              for (int i = 0; i < CH; ++i) {
+                const int64_t m = m0 + i;
+                if (m < p.M) store_out(p, m, n, (int32_t)r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"((uint32_t)L::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// Sums the split-K int32 partials in split order (exact) and applies the epilogue.
+__global__ void __launch_bounds__(256)
+splitk_reduce_kernel(const int32_t* __restrict__ ws, int splits, int64_t M, int64_t N, const float* __restrict__ sx,
+                     const float* __restrict__ sw, void* __restrict__ y, int64_t ldy, int ydt) {
+  const int64_t total = M * N;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    int32_t acc = 0;
+    for (int s = 0; s < splits; ++s) acc += ws[(int64_t)s * total + i];
+    const int64_t m = i / N, n = i % N;
+    const int64_t off = m * ldy + n;
+    if (ydt == SQ_BF16)
+      reinterpret_cast<__nv_bfloat16*>(y)[off] = __float2bfloat16_rn(dequant(acc, __ldg(sx + m), __ldg(sw + n)));
+    else if (ydt == SQ_F32)
+      reinterpret_cast<float*>(y)[off] = dequant(acc, __ldg(sx + m), __ldg(sw + n));
+    else
+      reinterpret_cast<int32_t*>(y)[off] = acc;
+  }
+}
+
+}  // namespace sqk
+
+// ============================================================================= host side
+namespace sqh {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D int8 tensor [rows, K] (K contiguous) tiled as box_rows x 128 bytes, 128-byte swizzle,
+// zero fill outside the tensor.
+static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {(cuuint32_t)sqk::BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launch plan for one GEMM shape on the current device.
+struct GemmPlan {
+  bool swap;
+  int bn;
+  int tiles_a, tiles_b, num_kb, kb_per_split, splits;
+  size_t ws_bytes;
+};
+
+static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
+  GemmPlan pl{};
+  const int sms = num_sms();
+  pl.swap = M <= 128;
+  if (pl.swap) {
+    pl.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    pl.tiles_a = (int)((N + sqk::BM - 1) / sqk::BM);
+    pl.tiles_b = 1;
+  } else {
+    pl.bn = 256;
+    pl.tiles_a = (int)((M + sqk::BM - 1) / sqk::BM);
+    pl.tiles_b = (int)((N + pl.bn - 1) / pl.bn);
+  }
+  pl.num_kb = (int)((K + sqk::BK - 1) / sqk::BK);
+  const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
+  int splits = 1;
+  if (tiles < sms) {
+    splits = (int)std::max<int64_t>(1, sms / tiles);
+    splits = std::min(splits, std::max(1, pl.num_kb / 4));
+  }
+  pl.kb_per_split = (pl.num_kb + splits - 1) / splits;
+  pl.splits = (pl.num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
+  pl.ws_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(int32_t) : 0;
+  return pl;
+}
+
+size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K) { return plan_gemm(M, N, K).ws_bytes; }
+
+template <int BN, int STAGES, bool SWAP>
+static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const sqk::GemmParams& p,
+                              cudaStream_t st) {
+  using L = sqk::GemmSmem<BN, STAGES>;
+  auto kern = sqk::w8a8_gemm_kernel<BN, STAGES, SWAP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(p.num_units, num_sms());
+  kern<<<grid, sqk::GEMM_THREADS, L::TOTAL, st>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
+                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
+                        bool* ws_too_small) {
+  const GemmPlan pl = plan_gemm(M, N, K);
+  *ws_too_small = pl.ws_bytes > 0 && (ws == nullptr || ws_bytes < pl.ws_bytes);
+  if (*ws_too_small) return cudaSuccess;
+  CUtensorMap ma, mb;
+  const void* a_ptr = pl.swap ? (const void*)wq : (const void*)xq;
+  const void* b_ptr = pl.swap ? (const void*)xq : (const void*)wq;
+  const int64_t a_rows = pl.swap ? N : M;
+  const int64_t b_rows = pl.swap ? M : N;
+  if (!make_map(&ma, a_ptr, a_rows, K, sqk::BM) || !make_map(&mb, b_ptr, b_rows, K, pl.bn))
+    return cudaErrorInvalidValue;
+  sqk::GemmParams p{};
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.num_kb = pl.num_kb;
+  p.kb_per_split = pl.kb_per_split;
+  p.splits = pl.splits;
+  p.num_units = pl.tiles_a * pl.tiles_b * pl.splits;
+  p.group_a = pl.swap ? 1 : 16;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.sx = sx;
+  p.sw = sw;
+  p.y = y;
+  p.ldy = ldy;
+  p.ydt = ydt;
+  const int64_t elt = ydt == SQ_BF16 ? 2 : 4;
+  p.vec_store = (reinterpret_cast<uintptr_t>(y) % 16 == 0) && (ldy * elt) % 16 == 0;
+  p.ws = static_cast<int32_t*>(ws);
+  cudaError_t e;
+  if (!pl.swap) {
+    e = launch_cfg<256, 4, false>(ma, mb, p, st);
+  } else {
+    switch (pl.bn) {
+      case 16: e = launch_cfg<16, 10, true>(ma, mb, p, st); break;
+      case 32: e = launch_cfg<32, 9, true>(ma, mb, p, st); break;
+      case 64: e = launch_cfg<64, 8, true>(ma, mb, p, st); break;
+      default: e = launch_cfg<128, 6, true>(ma, mb, p, st); break;
+    }
+  }
+  if (e != cudaSuccess || pl.splits == 1) return e;
+  const int64_t total = M * N;
+  const int64_t grid = std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 16);
+  sqk::splitk_reduce_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const int32_t*>(ws), pl.splits, M, N, sx,
+                                                            sw, y, ldy, ydt);
+  return cudaGetLastError();
+}
+
+cudaError_t read_device_error(unsigned int* code, int clear, cudaStream_t st) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(code, sqk::g_error_word, sizeof(unsigned int), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess || !clear) return e;
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(sqk::g_error_word, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);
+}
+
+}  // namespace sqh
