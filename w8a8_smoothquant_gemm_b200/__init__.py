@@ -152,7 +152,8 @@ def sq_smooth_factors(ax: torch.Tensor, aw: torch.Tensor, alpha: float, out: tor
 
 def sq_fold_quant_weights(W: torch.Tensor, s: torch.Tensor, gamma: torch.Tensor | None = None,
                           beta: torch.Tensor | None = None, wq: torch.Tensor | None = None,
-                          sw: torch.Tensor | None = None, stream=None):
+                          sw: torch.Tensor | None = None, gamma_f: torch.Tensor | None = None,
+                          beta_f: torch.Tensor | None = None, stream=None):
     """W [K, N] -> (Wq [N, K] int8, sw [N], gamma / s or None, beta / s or None)."""
     W = _mat(W, "W")
     K, N = W.shape
@@ -164,8 +165,11 @@ def sq_fold_quant_weights(W: torch.Tensor, s: torch.Tensor, gamma: torch.Tensor 
         wq = torch.empty(N, K, dtype=torch.int8, device=dev)
     if sw is None:
         sw = torch.empty(N, dtype=torch.float32, device=dev)
-    gf = torch.empty(K, dtype=torch.float32, device=dev) if gamma is not None else None
-    bf = torch.empty(K, dtype=torch.float32, device=dev) if beta is not None else None
+    gf = bf = None
+    if gamma is not None:
+        gf = gamma_f if gamma_f is not None else torch.empty(K, dtype=torch.float32, device=dev)
+    if beta is not None:
+        bf = beta_f if beta_f is not None else torch.empty(K, dtype=torch.float32, device=dev)
     _check("sq_fold_quant_weights",
            lib().sq_fold_quant_weights(_ptr(W), _dt(W), K, N, W.stride(0), _ptr(s), _ptr(gamma), _ptr(beta),
                                        _ptr(wq), _ptr(sw), _ptr(gf), _ptr(bf), _stream(stream)))

@@ -205,7 +205,7 @@ static cudaError_t launch_calib_ln_t(const void* x, int64_t rows, int K, int64_t
   const bool rows_atomic = smem_cols > 160 * 1024;
   const size_t smem = rows_atomic ? 0 : smem_cols;
   auto kern = sqk::calib_ln_absmax_kernel<BF16, MAXC>;
-  if (smem > 48 * 1024) {
+  {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
