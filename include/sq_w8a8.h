@@ -139,6 +139,30 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, cons
  * launch it picks does not split K).  Returns (size_t)-1 for invalid sizes. */
 size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
+/* Size of the scratch array behind sq_w8a8_gemm_noalloc (16 MiB). */
+#define SQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* sq_w8a8_gemm_noalloc -- sq_w8a8_gemm for callers that cannot allocate device memory.
+ *   The pages have no counterpart: this is a library convenience.  Some callers must not
+ *   call cudaMalloc: a plug-in inside a host program that owns all device memory through
+ *   its own pool (an allocation would fail or break that program's accounting), or a
+ *   latency-critical loop where cudaMalloc may synchronise the device.  This variant takes
+ *   no workspace: when the launch splits K, its int32 partial sums go to a scratch array of
+ *   SQ_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads the
+ *   library holds until the process exits.  The caller still passes all inputs and
+ *   outputs, with the same meaning, layout and checks as sq_w8a8_gemm.
+ *   - A shape whose workspace (sq_w8a8_gemm_workspace_size) exceeds the scratch returns
+ *     SQ_ERR_WORKSPACE with nothing launched.
+ *   - The first call on a device looks up the scratch array's device address (set-up, once
+ *     per device, with that device current); make that first call before any stream
+ *     capture.  A failed look-up returns SQ_ERR_CUDA.
+ *   - Every call on a device shares the one array, which keeps the last call's contents;
+ *     each call overwrites the partial sums it reads, so nothing needs to start at zero.
+ *     Calls that overlap on the GPU (different streams, no ordering) race on it. */
+sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                               int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
+                               void* stream);
+
 /* Reads (and with clear != 0 resets) the device-side error word of the current device:
  * 0 when no kernel gave up on a bounded wait.  Synchronises `stream`. */
 sq_status sq_device_error(unsigned int* code, int clear, void* stream);
