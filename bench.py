@@ -421,29 +421,46 @@ def run_device(args, rank, world, local):
 
 
 def run_kernel(args):
-    """One kernel of the path on one shape, `--steps` times (for profiler captures)."""
+    """One kernel of the path on one shape, `--steps` times, CUDA-event timed (profiling aid).
+
+    --shape M,N,K; the activation is [M, K] with a LayerNorm in front, the weight [K, N]."""
     import w8a8_smoothquant_gemm_b200 as sq
     M, N, K = (int(v) for v in args.shape.split(","))
     device = torch.device("cuda", 0)
     L = Linear("k", K, N, True, M, device, 7)
     L.run(sq, 1)
     torch.cuda.synchronize()
-    for _ in range(args.steps):
-        if args.kernel == "gemm":
-            sq.sq_w8a8_gemm(L.xq, L.sx, L.wq, L.sw, y=L.y, workspace=L.ws)
-        elif args.kernel == "fold":
-            sq.sq_fold_quant_weights(L.W, L.s, L.gamma, wq=L.wq, sw=L.sw, gamma_f=L.gf)
-        elif args.kernel == "lnquant":
-            sq.sq_ln_smooth_quant(L.x, gamma_f=L.gf, xq=L.xq, sx=L.sx)
-        elif args.kernel == "calib":
-            sq.sq_calib_ln_absmax(L.x, L.gamma, out=L.ax)
-        elif args.kernel == "wabsmax":
-            sq.sq_calib_absmax(L.W, 1, out=L.aw)
-        elif args.kernel == "xabsmax":
-            sq.sq_calib_absmax(L.x, 0, out=L.ax)
+    calls = {
+        "gemm": (lambda: sq.sq_w8a8_gemm(L.xq, L.sx, L.wq, L.sw, y=L.y, workspace=L.ws),
+                 M * K + N * K + 2 * M * N + 4 * (M + N), 2.0 * M * N * K),
+        "fold": (lambda: sq.sq_fold_quant_weights(L.W, L.s, L.gamma, wq=L.wq, sw=L.sw, gamma_f=L.gf),
+                 L.bytes_fold(), 0.0),
+        "lnquant": (lambda: sq.sq_ln_smooth_quant(L.x, gamma_f=L.gf, xq=L.xq, sx=L.sx), L.bytes_quant(), 0.0),
+        "quant": (lambda: sq.sq_ln_smooth_quant(L.x, s=L.s, xq=L.xq, sx=L.sx), L.bytes_quant(), 0.0),
+        "calib": (lambda: sq.sq_calib_ln_absmax(L.x, L.gamma, out=L.ax), L.bytes_calib(), 0.0),
+        "xabsmax": (lambda: sq.sq_calib_absmax(L.x, 0, out=L.ax), M * K * 2 + 4 * K, 0.0),
+        "wabsmax": (lambda: sq.sq_calib_absmax(L.W, 1, out=L.aw), L.bytes_wabsmax(), 0.0),
+    }
+    fn, nbytes, ops = calls[args.kernel]
+    for _ in range(args.warmup):
+        fn()
     torch.cuda.synchronize()
-    print(json.dumps({"kernel": args.kernel, "shape": [M, N, K], "steps": args.steps,
-                      "device_error": sq.sq_device_error(clear=True)}))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(b) / 1e3 for a, b in evs)
+    med = t[len(t) // 2]
+    peaks = load_peaks()
+    out = {"kernel": args.kernel, "shape": [M, N, K], "steps": args.steps, "median_us": round(med * 1e6, 2),
+           "gbs": round(nbytes / med / 1e9, 1), "hbm_frac": round(nbytes / med / 1e9 / peaks["hbm_gbs"], 3),
+           "device_error": sq.sq_device_error(clear=True)}
+    if ops:
+        out["tops"] = round(ops / med / 1e12, 1)
+        out["int8_frac"] = round(ops / med / 1e12 / (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
+    print(json.dumps(out), flush=True)
 
 
 def main():
@@ -453,7 +470,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=("gemm", "fold", "lnquant", "calib", "wabsmax", "xabsmax"),
+    ap.add_argument("--kernel", choices=("gemm", "fold", "lnquant", "quant", "calib", "wabsmax", "xabsmax"),
                     help="run only this kernel on --shape M,N,K (profiling aid; prints no bench line)")
     ap.add_argument("--shape", default="2048,4096,4096")
     args = ap.parse_args()

@@ -136,6 +136,8 @@ def test_smooth_factors(alpha):
 @pytest.mark.parametrize("K,N,extra", [(16, 8, 0), (256, 256, 0), (272, 200, 8), (4096, 4096, 0), (1040, 3000, 0)])
 def test_fold_quant_weights(dt, K, N, extra):
     c = sq_inputs.make_case(4, K, N, K + N, x_dtype=dt, w_dtype=dt, beta_std=0.1)
+    if N > 3:
+        c.W[:, 3] = 0  # an all-zero output channel: scale 0, codes 0
     rng = np.random.default_rng(K)
     s = np.exp(rng.uniform(-2, 3, K)).astype(np.float32)
     Wh = padded(c.W, extra)
@@ -160,7 +162,8 @@ def test_fold_full_size(K, N):
 
 # ----------------------------------------------------------------------------- LN + smooth + quant
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
-@pytest.mark.parametrize("M,K", [(1, 16), (5, 256), (64, 4096), (3, 12288), (17, 14336), (2, 49152)])
+@pytest.mark.parametrize("M,K", [(1, 16), (5, 256), (9, 1040), (33, 2048), (64, 4096), (7, 8192), (3, 12288),
+                                 (17, 14336), (4, 16384), (3, 16400), (2, 49152)])
 @pytest.mark.parametrize("mode", ["ln", "plain"])
 def test_ln_smooth_quant(dt, M, K, mode):
     if dt == "f32" and K > 32768:
@@ -184,7 +187,7 @@ def test_ln_smooth_quant(dt, M, K, mode):
     assert np.array_equal(host(xq), r_xq)
 
 
-@pytest.mark.parametrize("rows,K", [(1, 256), (100, 4096), (1000, 4096), (33, 49152)])
+@pytest.mark.parametrize("rows,K", [(1, 256), (100, 4096), (1000, 4096), (70, 8192), (5, 14336), (33, 49152)])
 def test_calib_ln_absmax(rows, K):
     c = sq_inputs.make_case(rows, K, 8, rows + K, beta_std=0.1)
     got = sq.sq_calib_ln_absmax(dev(c.x), dev(c.gamma), dev(c.beta))

@@ -125,10 +125,10 @@ absmax_rows_kernel(const char* __restrict__ x, int64_t rows, int64_t nvec, int64
 
 // ---------------------------------------------------------------------------- LayerNorm output
 // Blocks loop over rows; each thread keeps the running max of the elements of its own
-// chunks in shared memory (no conflicts), then one atomicMax per column per block.
-// With rows_atomic set (K too large for shared memory) the running max goes straight
-// to global memory with an atomic per element per row.
-template <bool BF16, int MAXC>
+// chunks -- in registers (REG, rows of up to 32 elements per thread) or in shared memory --
+// then one atomicMax per column per block.  With rows_atomic set (K too large for shared
+// memory) the running max goes straight to global memory with an atomic per element per row.
+template <bool BF16, int MAXC, bool PREFETCH, bool REG>
 __global__ void __launch_bounds__(ROW_THREADS)
 calib_ln_absmax_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t ld_bytes,
                        const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
@@ -136,11 +136,19 @@ calib_ln_absmax_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t 
   extern __shared__ float colmax[];
   __shared__ float red[2 * (ROW_WARPS + 1)];
   const int nchunks = K / 8;
-  if (!rows_atomic)
+  float cm[REG ? MAXC * 8 : 1];
+  if (REG) {
+#pragma unroll
+    for (int i = 0; i < MAXC * 8; ++i) cm[i] = 0.0f;
+  } else if (!rows_atomic) {
     for (int j = threadIdx.x; j < K; j += ROW_THREADS) colmax[j] = 0.0f;
+  }
+  RowChunks<BF16, MAXC> rc;
+  if ((int64_t)blockIdx.x < rows) rc.load(x + (int64_t)blockIdx.x * ld_bytes, nchunks);
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    RowChunks<BF16, MAXC> rc;
-    rc.load(x + r * ld_bytes, nchunks);
+    const int64_t rn = r + gridDim.x;
+    RowChunks<BF16, MAXC> nxt;
+    if (PREFETCH && rn < rows) nxt.load(x + rn * ld_bytes, nchunks);
     float mu, rstd;
     row_stats(rc, nchunks, K, eps, red, mu, rstd);
 #pragma unroll
@@ -152,15 +160,75 @@ calib_ln_absmax_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t 
         ln_chunk(f, mu, rstd, gamma, beta, c, y);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          if (rows_atomic) atomic_max_nonneg(out + c * 8 + e, fabsf(y[e]));
+          if (REG) cm[i * 8 + e] = fmaxf(cm[i * 8 + e], fabsf(y[e]));
+          else if (rows_atomic) atomic_max_nonneg(out + c * 8 + e, fabsf(y[e]));
           else colmax[c * 8 + e] = fmaxf(colmax[c * 8 + e], fabsf(y[e]));
         }
       }
     }
+    if (PREFETCH) rc = nxt;
+    else if (rn < rows) rc.load(x + rn * ld_bytes, nchunks);
   }
-  if (!rows_atomic) {
+  if (REG) {
+    if ((int64_t)blockIdx.x < rows) {
+#pragma unroll
+      for (int i = 0; i < MAXC; ++i) {
+        const int c = threadIdx.x + i * ROW_THREADS;
+        if (c < nchunks)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) atomic_max_nonneg(out + c * 8 + e, cm[i * 8 + e]);
+      }
+    }
+  } else if (!rows_atomic) {
     __syncthreads();
     for (int j = threadIdx.x; j < K; j += ROW_THREADS) atomic_max_nonneg(out + j, colmax[j]);
+  }
+}
+
+// Rows of up to 8192 elements: one group of T threads per row (see sq_rowln.cuh), the
+// running column max of the thread's own chunks in registers across all rows the group
+// visits, one atomicMax per column per group at the end.
+template <bool BF16, int T, int NCH>
+__global__ void __launch_bounds__(256)
+calib_ln_group_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t ld_bytes,
+                      const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                      float* __restrict__ out) {
+  constexpr int G = 256 / T;
+  __shared__ float red[G][16];
+  const int gid = threadIdx.x / T, t = threadIdx.x % T;
+  const int nchunks = K / 8;
+  float cm[NCH * 8];
+#pragma unroll
+  for (int i = 0; i < NCH * 8; ++i) cm[i] = 0.0f;
+  RowRaw<BF16, NCH> raw;
+  const int64_t rstep = (int64_t)gridDim.x * G;
+  const int64_t r0 = (int64_t)blockIdx.x * G + gid;
+  if (r0 < rows) raw.template load<T>(x + r0 * ld_bytes, nchunks, t);
+  for (int64_t r = r0; r < rows; r += rstep) {
+    float v[NCH * 8];
+    raw.to_float(v);
+    if (r + rstep < rows) raw.template load<T>(x + (r + rstep) * ld_bytes, nchunks, t);
+    float mu, rstd;
+    group_row_stats<T, NCH>(v, nchunks, K, eps, red[gid], t, gid, mu, rstd);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = t + T * i;
+      if (c < nchunks) {
+        float y[8];
+        ln_chunk(v + i * 8, mu, rstd, gamma, beta, c, y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cm[i * 8 + e] = fmaxf(cm[i * 8 + e], fabsf(y[e]));
+      }
+    }
+  }
+  if (r0 < rows) {
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = t + T * i;
+      if (c < nchunks)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) atomic_max_nonneg(out + c * 8 + e, cm[i * 8 + e]);
+    }
   }
 }
 
@@ -201,10 +269,11 @@ cudaError_t launch_absmax(const void* x, bool bf16, int64_t rows, int64_t cols, 
 template <bool BF16, int MAXC>
 static cudaError_t launch_calib_ln_t(const void* x, int64_t rows, int K, int64_t ld_bytes, const float* gamma,
                                      const float* beta, float eps, float* out, cudaStream_t st) {
+  constexpr bool REG = MAXC <= 4;
   const size_t smem_cols = sizeof(float) * (size_t)K;
-  const bool rows_atomic = smem_cols > 160 * 1024;
-  const size_t smem = rows_atomic ? 0 : smem_cols;
-  auto kern = sqk::calib_ln_absmax_kernel<BF16, MAXC>;
+  const bool rows_atomic = !REG && smem_cols > 160 * 1024;
+  const size_t smem = (REG || rows_atomic) ? 0 : smem_cols;
+  auto kern = sqk::calib_ln_absmax_kernel<BF16, MAXC, BF16 && MAXC <= 4, REG>;
   {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -218,6 +287,34 @@ static cudaError_t launch_calib_ln_t(const void* x, int64_t rows, int K, int64_t
   return cudaGetLastError();
 }
 
+int pick_row_threads(int64_t K, int max_nch, int* nch);
+bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch);
+cudaError_t launch_rowpipe_calib(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx, const float* gamma,
+                                 const float* beta, float eps, float* out, int T, int nch, cudaStream_t st);
+
+template <bool BF16, int T, int NCH>
+static cudaError_t launch_calib_group_t(const void* x, int64_t rows, int K, int64_t ld_bytes, const float* gamma,
+                                        const float* beta, float eps, float* out, cudaStream_t st) {
+  auto kern = sqk::calib_ln_group_kernel<BF16, T, NCH>;
+  int per_sm = 1;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+  if (e != cudaSuccess) return e;
+  constexpr int G = 256 / T;
+  const int64_t blocks = (rows + G - 1) / G;
+  const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
+  kern<<<(unsigned)grid, 256, 0, st>>>((const char*)x, rows, K, ld_bytes, gamma, beta, eps, out);
+  return cudaGetLastError();
+}
+
+template <bool BF16, int T>
+static cudaError_t launch_calib_group_nch(int nch, const void* x, int64_t rows, int K, int64_t ld_bytes,
+                                          const float* gamma, const float* beta, float eps, float* out,
+                                          cudaStream_t st) {
+  if (nch <= 1) return launch_calib_group_t<BF16, T, 1>(x, rows, K, ld_bytes, gamma, beta, eps, out, st);
+  if (nch <= 2) return launch_calib_group_t<BF16, T, 2>(x, rows, K, ld_bytes, gamma, beta, eps, out, st);
+  return launch_calib_group_t<BF16, T, 4>(x, rows, K, ld_bytes, gamma, beta, eps, out, st);
+}
+
 cudaError_t launch_calib_ln_absmax(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ld,
                                    const float* gamma, const float* beta, float eps, int accumulate,
                                    float* out, cudaStream_t st) {
@@ -226,6 +323,20 @@ cudaError_t launch_calib_ln_absmax(const void* x, bool bf16, int64_t rows, int64
     if (e != cudaSuccess) return e;
   }
   const int64_t ldb = ld * (bf16 ? 2 : 4);
+  int pT = 0, pn = 0;
+  if (rowpipe_shape(K, bf16, 4, &pT, &pn))
+    return launch_rowpipe_calib(x, bf16, rows, K, ld, gamma, beta, eps, out, pT, pn, st);
+  int gnch = 0;
+  const int T = pick_row_threads(K, 4, &gnch);
+  if (T) {
+    const int k = (int)K;
+#define SQ_T(TT)                                                                                       \
+  if (T == TT)                                                                                         \
+    return bf16 ? launch_calib_group_nch<true, TT>(gnch, x, rows, k, ldb, gamma, beta, eps, out, st)   \
+                : launch_calib_group_nch<false, TT>(gnch, x, rows, k, ldb, gamma, beta, eps, out, st);
+    SQ_T(32) SQ_T(64) SQ_T(128) SQ_T(256)
+#undef SQ_T
+  }
   const int need = (int)((K / 8 + sqk::ROW_THREADS - 1) / sqk::ROW_THREADS);
   const int k = (int)K;
 #define SQ_LN_CASE(C)                                                                                   \

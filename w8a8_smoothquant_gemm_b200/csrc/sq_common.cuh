@@ -19,6 +19,8 @@ enum : unsigned int {
   ERR_GEMM_PRODUCER_WAIT = 1u << 0,
   ERR_GEMM_MMA_WAIT = 1u << 1,
   ERR_GEMM_EPILOGUE_WAIT = 1u << 2,
+  ERR_FOLD_TMA_WAIT = 1u << 3,
+  ERR_ROW_TMA_WAIT = 1u << 4,
 };
 
 // bf16 bits -> fp32 (exact widening).
@@ -38,6 +40,49 @@ __device__ __forceinline__ int quant_code(float v, float scale) {
   if (scale == 0.0f) return 0;
   int q = __float2int_rn(__fdiv_rn(v, scale));
   return max(-127, min(127, q));
+}
+
+// Division by a divisor shared by many dividends (a per-row or per-column scale).
+// Markstein's theorem (P. Markstein, IBM J. Res. Dev. 34(1), 1990; Muller et al., Handbook
+// of Floating-Point Arithmetic, sec. on division with FMA): with y = RN(1/b) and
+// q = RN(a * y), the remainder r = a - b q is exact under FMA and RN(q + r y) is the
+// correctly rounded a / b, barring underflow or overflow of the intermediates.
+struct SharedDivisor {
+  float b, y;
+  bool fast;  // b is far from the subnormal range, so the intermediates stay normal
+  // A zero divisor (all-zero row or column) is turned into "multiply by 0", so every code
+  // of that row or column is 0, as the quantiser defines.
+  __device__ __forceinline__ explicit SharedDivisor(float b_) : b(b_) {
+    if (b_ == 0.0f) {
+      b = 1.0f;
+      y = 0.0f;
+      fast = true;
+      return;
+    }
+    fast = fabsf(b_) >= 0x1p-90f && fabsf(b_) <= 0x1p+90f;
+    y = fast ? __frcp_rn(b_) : 0.0f;
+  }
+  __device__ __forceinline__ float div(float a) const {
+    if (!fast) return __fdiv_rn(a, b);
+    const float q = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(r, y, q);
+  }
+};
+
+// Code of v with a shared scale, returned in the low byte of a 32-bit word: the
+// correctly rounded quotient q = v / scale satisfies |q| <= 127 (1 + 2^-23) because
+// |v| <= absmax and scale = RN(absmax / 127), so adding 1.5 * 2^23 rounds q to the nearest
+// integer, ties to even (the float grid has spacing 1 there), and leaves rne(q) mod 256 in
+// the low byte of the sum's bit pattern.  The clamp to [-127, 127] can never bind.
+// A zero scale gives code 0 (see SharedDivisor).
+__device__ __forceinline__ uint32_t code_bits(float v, const SharedDivisor& d) {
+  return __float_as_uint(__fadd_rn(d.div(v), 12582912.0f));
+}
+
+// Low bytes of four words -> one packed word (first argument in the low byte).
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // Packs four codes (low byte first) into one 32-bit word.
@@ -64,6 +109,6 @@ __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
 
 // Host-side launch helpers (internal to the library; no C ABI).
 namespace sqh {
-int num_sms();                 // SM count of the current device (cached per device)
-size_t max_smem_optin();       // opt-in shared memory per block of the current device
+int num_sms();                    // SM count of the current device (cached per device)
+unsigned int* error_word_ptr();   // device address of the error word (current device)
 }  // namespace sqh

@@ -11,7 +11,7 @@
 // through shared memory into Wq[N, K] (K contiguous), the GEMM's K-major operand.
 #include <algorithm>
 
-#include "sq_common.cuh"
+#include "sq_ptx.cuh"
 
 namespace sqk {
 
@@ -156,6 +156,125 @@ fold_quant_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_
   }
 }
 
+// ---------------------------------------------------------------------------- cluster fold
+// One thread-block cluster of C CTAs per strip of CW output channels.  CTA r of the
+// cluster owns rows [r * RK, (r + 1) * RK) of W (input channels): one thread TMA-loads that
+// RK x CW block into shared memory (W crosses HBM once), the CTA reduces its partial
+// column maxima of |s_j W_jk|, the C partials are combined through distributed shared
+// memory, and the CTA quantises its block from shared memory, writing Wq[k, j] transposed
+// (each thread emits 64 consecutive j of one k).  Rows beyond K and columns beyond N are
+// zero-filled by TMA and never stored.
+template <int CW>
+__global__ void __launch_bounds__(256)
+fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t N, int RK, int C,
+                    const float* __restrict__ s, const float* __restrict__ gamma, const float* __restrict__ beta,
+                    int8_t* __restrict__ Wq, float* __restrict__ sw, float* __restrict__ gamma_f,
+                    float* __restrict__ beta_f, unsigned int* err) {
+  constexpr int G = 256 / (CW / 8);  // row lanes of the max pass (8 columns per thread)
+  extern __shared__ uint8_t smem_raw[];
+  // TMA destinations want 128-byte alignment: round the dynamic base up (128 bytes of slack)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint16_t* tile = reinterpret_cast<const uint16_t*>(smem);      // [RK][CW] bf16 bits
+  float* s_rows = reinterpret_cast<float*>(smem + (size_t)RK * CW * 2);  // [RK]
+  __shared__ float red[G][CW + 1];
+  __shared__ float part[CW];
+  __shared__ float scale[CW];
+  __shared__ __align__(8) uint64_t bar;
+
+  const int tid = threadIdx.x;
+  const uint32_t crank = cluster_ctarank();
+  const int64_t strip = blockIdx.x / C;
+  const int64_t k0 = strip * CW;
+  const int64_t j0 = (int64_t)crank * RK;
+
+  for (int64_t j = (int64_t)blockIdx.x * 256 + tid; j < K; j += (int64_t)gridDim.x * 256) {
+    const float sj = s[j];
+    if (gamma && gamma_f) gamma_f[j] = __fdiv_rn(gamma[j], sj);
+    if (beta && beta_f) beta_f[j] = __fdiv_rn(beta[j], sj);
+  }
+
+  const uint32_t b = smem_u32(&bar);
+  if (tid == 0) {
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(b, (uint32_t)RK * CW * 2);
+    for (int r = 0; r < RK; r += 64) tma_load_2d(smem_u32(smem + (size_t)r * CW * 2), &wmap, b, (int)k0, (int)(j0 + r));
+  }
+  for (int i = tid; i < RK; i += 256) s_rows[i] = (j0 + i < K) ? __ldg(s + j0 + i) : 0.0f;
+  if (!mbar_wait(b, 0)) atomicOr(err, ERR_FOLD_TMA_WAIT);
+  __syncthreads();
+
+  // ---- partial column max of |s_j W_jk| over this CTA's rows: thread = 8 columns x rows rl + G m
+  {
+    const int cg = tid % (CW / 8), rl = tid / (CW / 8);
+    float m[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = 0.0f;
+    for (int j = rl; j < RK; j += G) {
+      const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
+      const float sj = s_rows[j];
+      float f[8];
+      unpack8_bf16(w, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(sj, f[e])));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
+  }
+  __syncthreads();
+  if (tid < CW) {
+    float m = red[0][tid];
+    for (int g = 1; g < G; ++g) m = fmaxf(m, red[g][tid]);
+    part[tid] = m;
+  }
+  cluster_sync();
+  if (tid < CW) {
+    float m = 0.0f;
+    for (int r = 0; r < C; ++r) m = fmaxf(m, ld_dsmem_f32(&part[tid], (uint32_t)r));
+    const float sc = __fdiv_rn(m, 127.0f);
+    scale[tid] = sc;
+    if (crank == 0 && k0 + tid < N) sw[k0 + tid] = sc;
+  }
+  __syncthreads();
+
+  // ---- codes, transposed: item = (4 adjacent columns, 16 consecutive rows); each item
+  // reads 16 x 8 bytes of shared memory and writes 16 codes to each of 4 rows of Wq.
+  const int items = (CW / 4) * (RK / 16);
+  for (int it = tid; it < items; it += 256) {
+    const int kq = (it % (CW / 4)) * 4, jl = (it / (CW / 4)) * 16;
+    if (j0 + jl >= K) continue;  // K % 16 == 0: a 16-row block is all in or all out
+    const SharedDivisor d0(scale[kq]), d1(scale[kq + 1]), d2(scale[kq + 2]), d3(scale[kq + 3]);
+    uint32_t words[4][4];
+#pragma unroll
+    for (int g4 = 0; g4 < 4; ++g4) {
+      uint32_t b[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = jl + g4 * 4 + r;
+        const uint2 w = *reinterpret_cast<const uint2*>(tile + j * CW + kq);
+        const float sj = s_rows[j];
+        b[0][r] = code_bits(__fmul_rn(sj, bf16lo(w.x)), d0);
+        b[1][r] = code_bits(__fmul_rn(sj, bf16hi(w.x)), d1);
+        b[2][r] = code_bits(__fmul_rn(sj, bf16lo(w.y)), d2);
+        b[3][r] = code_bits(__fmul_rn(sj, bf16hi(w.y)), d3);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) words[c][g4] = pack4_low_bytes(b[c][0], b[c][1], b[c][2], b[c][3]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t k = k0 + kq + c;
+      if (k < N)
+        *reinterpret_cast<uint4*>(Wq + k * K + j0 + jl) = make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
+    }
+  }
+  cluster_sync();  // peers may still be reading `part` through distributed shared memory
+}
+
 }  // namespace sqk
 
 namespace sqh {
@@ -188,16 +307,71 @@ static cudaError_t launch_fold_t(const void* W, int64_t K, int64_t N, int64_t ld
   return cudaGetLastError();
 }
 
+template <int CW>
+static cudaError_t launch_fold_cluster_t(const void* W, int64_t K, int64_t N, int64_t ldw, int C, int RK,
+                                         const float* s, const float* gamma, const float* beta, int8_t* Wq,
+                                         float* sw, float* gamma_f, float* beta_f, cudaStream_t st) {
+  CUtensorMap map;
+  if (!make_tmap_2d(&map, true, W, N, K, ldw * 2, CW, 64, false)) return cudaErrorInvalidValue;
+  const size_t smem = 128 + (size_t)RK * CW * 2 + (size_t)RK * 4;
+  auto kern = sqk::fold_cluster_kernel<CW>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t strips = (N + CW - 1) / CW;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(strips * C));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, K, N, RK, C, s, gamma, beta, Wq, sw, gamma_f, beta_f, error_word_ptr());
+}
+
+// Cluster shape of the single-pass fold: the widest strip (CW) and smallest cluster (C)
+// whose per-CTA block fits `budget` bytes of shared memory.
+static bool fold_cluster_shape(int64_t K, size_t budget, int* cw, int* c, int* rk) {
+  for (int w : {64, 32, 16})
+    for (int cl : {1, 2, 4, 8, 16}) {
+      const int64_t rows = ((K + cl - 1) / cl + 63) / 64 * 64;
+      if ((size_t)rows * w * 2 + (size_t)rows * 4 <= budget) {
+        *cw = w;
+        *c = cl;
+        *rk = (int)rows;
+        return true;
+      }
+    }
+  return false;
+}
+
 cudaError_t launch_fold_quant(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
                               const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
                               float* beta_f, cudaStream_t st) {
+  int cw = 0, cl = 0, rk = 0;
+  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 &&
+      (fold_cluster_shape(K, 72 * 1024, &cw, &cl, &rk) || fold_cluster_shape(K, 200 * 1024, &cw, &cl, &rk))) {
+    switch (cw) {
+      case 64: return launch_fold_cluster_t<64>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      case 32: return launch_fold_cluster_t<32>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      default: return launch_fold_cluster_t<16>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+    }
+  }
   // narrower strips when there are few output channels, so every SM gets work
   const int64_t sms = num_sms();
-  const int cw = (N / 32 >= 2 * sms) ? 32 : 16;
+  const int strip = (N / 32 >= 2 * sms) ? 32 : 16;
   if (bf16)
-    return cw == 32 ? launch_fold_t<true, 32>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
+    return strip == 32 ? launch_fold_t<true, 32>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
                     : launch_fold_t<true, 16>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-  return cw == 32 ? launch_fold_t<false, 32>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
+  return strip == 32 ? launch_fold_t<false, 32>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
                   : launch_fold_t<false, 16>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
 }
 

@@ -28,8 +28,9 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
 
-#include "sq_common.cuh"
+#include "sq_ptx.cuh"
 
 namespace sqk {
 
@@ -39,7 +40,6 @@ constexpr int BM = 128;          // MMA M: rows of the A operand per tile
 constexpr int BK = 128;          // K bytes per ring stage (one 128-byte swizzle row)
 constexpr int UMMA_K = 32;       // K per tcgen05.mma kind::i8
 constexpr int GEMM_THREADS = 192;
-constexpr unsigned long long WAIT_NS = 10ull * 1000 * 1000 * 1000;  // 10 s per wait
 
 struct GemmParams {
   int tiles_a, tiles_b;      // tiles along A rows (BM) and B rows (BN)
@@ -57,57 +57,24 @@ struct GemmParams {
   int32_t* ws;               // [splits][M][N] int32 partials when splits > 1
 };
 
-// ----------------------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
+// TMA load whose completion is signalled on the mbarrier of the pair's leader CTA
+// (`bar` is a shared::cluster address, e.g. from mapa).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Waits for the phase with the given parity to complete; false after `limit_ns`.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          unsigned long long limit_ns = WAIT_NS) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 0 && global_ns() - t0 > limit_ns) return false;
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -117,15 +84,33 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, int8 -> int32.
+// Arrives on the same mbarrier in both CTAs of the pair when this thread's MMAs complete.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(bar)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, int8 -> int32; CG = 2 spans the CTA pair
+// (M = 256, each CTA supplies 128 rows of A and half of B from the same smem offsets).
+template <int CG>
 __device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if (CG == 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major tile written by TMA with 128-byte
@@ -203,10 +188,13 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta,
   tb = in_group / ga;
 }
 
-template <int BN, int STAGES>
+// Shared-memory layout of one CTA: BN_CTA rows of B per stage (BN / CG), BN accumulator
+// columns per TMEM buffer.
+template <int BN, int STAGES, int CG>
 struct GemmSmem {
+  static constexpr int BN_CTA = BN / CG;
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
+  static constexpr int B_BYTES = BN_CTA * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 4;
@@ -214,13 +202,20 @@ struct GemmSmem {
   static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;  // power of two for BN in {16..256}
 };
 
-template <int BN, int STAGES, bool SWAP>
+// CG = 1: one CTA per output tile of 128 x BN.  CG = 2: a cluster of two CTAs per tile of
+// 256 x BN; CTA r loads rows [128 r, 128 r + 128) of the A tile and [BN/2 r, BN/2 (r+1)) of
+// the B tile, signalling the leader's (rank 0) full barrier; the leader issues the pair MMAs
+// and its commits arrive on the barriers of both CTAs; each CTA's epilogue drains its own
+// TMEM (its 128 rows x BN columns) and arrives on the leader's accumulator-empty barrier.
+template <int BN, int STAGES, bool SWAP, int CG>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const GemmParams p) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, CG>;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M = 128 needs N % 16 == 0, 16..256");
-  constexpr uint32_t IDESC = idesc_i8(BM, BN);
+  static_assert(CG == 1 || (!SWAP && BN % 32 == 0), "the pair path runs the non-swapped layout, N % 32 == 0");
+  constexpr int MMA_M = BM * CG;
+  constexpr uint32_t IDESC = idesc_i8(MMA_M, BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -232,6 +227,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::BAR_OFFSET + L::NUM_BARS * 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = blockIdx.x / CG, unit_step = gridDim.x / CG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -240,7 +238,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);
+      mbar_init(tempty_bar(a), 4 * CG);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -248,25 +246,33 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                 "r"((uint32_t)L::TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (CG == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                   "r"((uint32_t)L::TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                   "r"((uint32_t)L::TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync();  // the peer's loads signal the leader's barriers: init first
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer (each CTA)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       uint32_t issued = 0;  // bit s: stage s has been loaded; its last load used parity bit s of `par`
       uint32_t par = 0;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      for (int u = unit0; u < p.num_units && ok; u += unit_step) {
         int ta, tb, split;
         decode_unit(p, u, ta, tb, split);
         const int kb0 = split * p.kb_per_split;
@@ -279,30 +285,37 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           }
           issued |= 1u << stage;
           par = (par & ~(1u << stage)) | (phase << stage);
-          mbar_arrive_expect_tx(full_bar(stage), (uint32_t)L::STAGE_BYTES);
           const uint32_t sa = sbase + stage * L::STAGE_BYTES;
-          tma_load_2d(sa, &map_a, full_bar(stage), kb * BK, ta * BM);
-          tma_load_2d(sa + L::A_BYTES, &map_b, full_bar(stage), kb * BK, tb * BN);
+          if (CG == 1) {
+            mbar_arrive_expect_tx(full_bar(stage), (uint32_t)L::STAGE_BYTES);
+            tma_load_2d(sa, &map_a, full_bar(stage), kb * BK, ta * BM);
+            tma_load_2d(sa + L::A_BYTES, &map_b, full_bar(stage), kb * BK, tb * BN);
+          } else {
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(CG * L::STAGE_BYTES));
+            const uint32_t fb = map_shared(full_bar(stage), 0);
+            tma_load_2d_pair(sa, &map_a, fb, kb * BK, ta * MMA_M + (int)rank * BM);
+            tma_load_2d_pair(sa + L::A_BYTES, &map_b, fb, kb * BK, tb * BN + (int)rank * L::BN_CTA);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (!ok) {
-        // let the loads this thread issued land before the block exits (bounded, 100 ms)
+      if (!ok && leader) {
+        // let the loads issued for this barrier land before the block exits (bounded, 100 ms)
         for (int s = 0; s < STAGES; ++s)
           if (issued & (1u << s)) (void)mbar_wait(full_bar(s), (par >> s) & 1u, 100ull * 1000 * 1000);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++it) {
+      for (int u = unit0; u < p.num_units && ok; u += unit_step, ++it) {
         int ta, tb, split;
         decode_unit(p, u, ta, tb, split);
         const int kb0 = split * p.kb_per_split;
@@ -326,24 +339,26 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           const uint32_t sb = sa + L::A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
-            tc_mma_i8(d_tmem, sw128_desc(sa + k * UMMA_K), sw128_desc(sb + k * UMMA_K), IDESC,
-                      (kb > kb0 || k > 0) ? 1u : 0u);
+            tc_mma_i8<CG>(d_tmem, sw128_desc(sa + k * UMMA_K), sw128_desc(sb + k * UMMA_K), IDESC,
+                          (kb > kb0 || k > 0) ? 1u : 0u);
           }
-          tc_commit(empty_bar(stage));
+          if (CG == 1) tc_commit(empty_bar(stage));
+          else tc_commit_pair(empty_bar(stage));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        tc_commit(tfull_bar(acc));
+        if (CG == 1) tc_commit(tfull_bar(acc));
+        else tc_commit_pair(tfull_bar(acc));
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;          // row of the A tile = TMEM lane
+    const int row = q * 32 + lane;          // row of this CTA's A tile = TMEM lane
     int it = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++it) {
+    for (int u = unit0; u < p.num_units; u += unit_step, ++it) {
       int ta, tb, split;
       decode_unit(p, u, ta, tb, split);
       const int acc = it & 1;
@@ -355,7 +370,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       __syncwarp();  // tcgen05.ld below is .sync.aligned: reconverge after the wait loop
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int64_t arow = (int64_t)ta * BM + row;
+      const int64_t arow = (int64_t)ta * MMA_M + (int64_t)rank * BM + row;
       constexpr int CH = BN >= 32 ? 32 : 16;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += CH) {
@@ -417,19 +432,30 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (lane == 0) {
+        if (CG == 1) mbar_arrive(tempty_bar(acc));
+        else mbar_arrive_cluster(map_shared(tempty_bar(acc), 0));
+      }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync();  // no CTA of the pair leaves while its peer may still use it
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"((uint32_t)L::TMEM_COLS)
-                 : "memory");
+    if (CG == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"((uint32_t)L::TMEM_COLS)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"((uint32_t)L::TMEM_COLS)
+                   : "memory");
   }
 }
+
 
 // Sums the split-K int32 partials in split order (exact) and applies the epilogue.
 __global__ void __launch_bounds__(256)
@@ -471,46 +497,67 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+bool make_tmap_2d(CUtensorMap* map, bool two_byte, const void* base, int64_t inner, int64_t outer,
+                  int64_t row_bytes, int box_inner, int box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, two_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D int8 tensor [rows, K] (K contiguous) tiled as box_rows x 128 bytes, 128-byte swizzle,
 // zero fill outside the tensor.
 static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)K};
-  cuuint32_t box[2] = {(cuuint32_t)sqk::BK, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tmap_2d(map, false, base, K, rows, K, sqk::BK, box_rows, true);
 }
 
 // Launch plan for one GEMM shape on the current device.
 struct GemmPlan {
   bool swap;
+  int cg;  // CTAs per MMA tile (2: a CTA pair computes 256-row tiles)
   int bn;
   int tiles_a, tiles_b, num_kb, kb_per_split, splits;
   size_t ws_bytes;
 };
 
+// Pair tiles unless SQ_GEMM_PAIR=0 is set in the environment (read once; a tuning aid).
+static bool pairs_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("SQ_GEMM_PAIR");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
   GemmPlan pl{};
   const int sms = num_sms();
   pl.swap = M <= 128;
+  pl.cg = 1;
   if (pl.swap) {
     pl.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
     pl.tiles_a = (int)((N + sqk::BM - 1) / sqk::BM);
     pl.tiles_b = 1;
   } else {
     pl.bn = 256;
-    pl.tiles_a = (int)((M + sqk::BM - 1) / sqk::BM);
+    pl.cg = pairs_enabled() ? 2 : 1;
+    const int64_t tile_m = (int64_t)sqk::BM * pl.cg;
+    pl.tiles_a = (int)((M + tile_m - 1) / tile_m);
     pl.tiles_b = (int)((N + pl.bn - 1) / pl.bn);
   }
   pl.num_kb = (int)((K + sqk::BK - 1) / sqk::BK);
   const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
+  const int slots = sms / pl.cg;  // tiles that run at once
   int splits = 1;
-  if (tiles < sms) {
-    splits = (int)std::max<int64_t>(1, sms / tiles);
+  if (tiles < slots) {
+    splits = (int)std::max<int64_t>(1, slots / tiles);
     splits = std::min(splits, std::max(1, pl.num_kb / 4));
   }
   pl.kb_per_split = (pl.num_kb + splits - 1) / splits;
@@ -521,16 +568,32 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K) { return plan_gemm(M, N, K).ws_bytes; }
 
-template <int BN, int STAGES, bool SWAP>
+template <int BN, int STAGES, bool SWAP, int CG>
 static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const sqk::GemmParams& p,
                               cudaStream_t st) {
-  using L = sqk::GemmSmem<BN, STAGES>;
-  auto kern = sqk::w8a8_gemm_kernel<BN, STAGES, SWAP>;
+  using L = sqk::GemmSmem<BN, STAGES, CG>;
+  auto kern = sqk::w8a8_gemm_kernel<BN, STAGES, SWAP, CG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
   if (e != cudaSuccess) return e;
-  const int grid = std::min(p.num_units, num_sms());
-  kern<<<grid, sqk::GEMM_THREADS, L::TOTAL, st>>>(ma, mb, p);
-  return cudaGetLastError();
+  const int slots = num_sms() / CG;
+  const int grid = std::min(p.num_units, slots) * CG;
+  if (CG == 1) {
+    kern<<<grid, sqk::GEMM_THREADS, L::TOTAL, st>>>(ma, mb, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(sqk::GEMM_THREADS);
+  cfg.dynamicSmemBytes = L::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
 }
 
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
@@ -544,7 +607,7 @@ cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, con
   const void* b_ptr = pl.swap ? (const void*)xq : (const void*)wq;
   const int64_t a_rows = pl.swap ? N : M;
   const int64_t b_rows = pl.swap ? M : N;
-  if (!make_map(&ma, a_ptr, a_rows, K, sqk::BM) || !make_map(&mb, b_ptr, b_rows, K, pl.bn))
+  if (!make_map(&ma, a_ptr, a_rows, K, sqk::BM) || !make_map(&mb, b_ptr, b_rows, K, pl.bn / pl.cg))
     return cudaErrorInvalidValue;
   sqk::GemmParams p{};
   p.tiles_a = pl.tiles_a;
@@ -553,7 +616,7 @@ cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, con
   p.kb_per_split = pl.kb_per_split;
   p.splits = pl.splits;
   p.num_units = pl.tiles_a * pl.tiles_b * pl.splits;
-  p.group_a = pl.swap ? 1 : 16;
+  p.group_a = pl.swap ? 1 : 16 / pl.cg;
   p.M = (int)M;
   p.N = (int)N;
   p.sx = sx;
@@ -566,13 +629,13 @@ cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, con
   p.ws = static_cast<int32_t*>(ws);
   cudaError_t e;
   if (!pl.swap) {
-    e = launch_cfg<256, 4, false>(ma, mb, p, st);
+    e = pl.cg == 2 ? launch_cfg<256, 6, false, 2>(ma, mb, p, st) : launch_cfg<256, 4, false, 1>(ma, mb, p, st);
   } else {
     switch (pl.bn) {
-      case 16: e = launch_cfg<16, 10, true>(ma, mb, p, st); break;
-      case 32: e = launch_cfg<32, 9, true>(ma, mb, p, st); break;
-      case 64: e = launch_cfg<64, 8, true>(ma, mb, p, st); break;
-      default: e = launch_cfg<128, 6, true>(ma, mb, p, st); break;
+      case 16: e = launch_cfg<16, 10, true, 1>(ma, mb, p, st); break;
+      case 32: e = launch_cfg<32, 9, true, 1>(ma, mb, p, st); break;
+      case 64: e = launch_cfg<64, 8, true, 1>(ma, mb, p, st); break;
+      default: e = launch_cfg<128, 6, true, 1>(ma, mb, p, st); break;
     }
   }
   if (e != cudaSuccess || pl.splits == 1) return e;
@@ -581,6 +644,18 @@ cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, con
   sqk::splitk_reduce_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const int32_t*>(ws), pl.splits, M, N, sx,
                                                             sw, y, ldy, ydt);
   return cudaGetLastError();
+}
+
+// Device address of the error word on the current device (for kernels in other files).
+unsigned int* error_word_ptr() {
+  static unsigned int* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, sqk::g_error_word) == cudaSuccess) ptrs[dev] = static_cast<unsigned int*>(p);
+  }
+  return ptrs[dev];
 }
 
 cudaError_t read_device_error(unsigned int* code, int clear, cudaStream_t st) {

@@ -15,49 +15,127 @@
 
 namespace sqk {
 
-template <bool BF16, int MAXC, bool LN>
+// Blocks loop over rows (grid sized to the resident blocks); with PREFETCH the next row's
+// loads are issued before the current row is reduced, so HBM stays busy during the
+// block-wide reductions.  With KEEP_Y the row's y values stay in registers between the
+// absmax and the quantisation (computed once); otherwise they are recomputed.
+template <bool BF16, int MAXC, bool LN, bool PREFETCH, bool KEEP_Y>
 __global__ void __launch_bounds__(ROW_THREADS)
 ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
                        const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
                        const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx) {
   __shared__ float red[3 * (ROW_WARPS + 1)];
   const int nchunks = K / 8;
-  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
-    RowChunks<BF16, MAXC> rc;
-    rc.load(x + m * ld_bytes, nchunks);
+  RowChunks<BF16, MAXC> cur;
+  int64_t m = blockIdx.x;
+  if (m < M) cur.load(x + m * ld_bytes, nchunks);
+  for (; m < M; m += gridDim.x) {
+    const int64_t mn = m + gridDim.x;
+    RowChunks<BF16, MAXC> nxt;
+    if (PREFETCH && mn < M) nxt.load(x + mn * ld_bytes, nchunks);
     float mu = 0.0f, rstd = 0.0f;
-    if (LN) row_stats(rc, nchunks, K, eps, red, mu, rstd);
-    // absmax of y
+    if (LN) row_stats(cur, nchunks, K, eps, red, mu, rstd);
+    float yk[KEEP_Y ? MAXC * 8 : 1];
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < MAXC; ++i) {
       const int c = threadIdx.x + i * ROW_THREADS;
       if (c < nchunks) {
         float f[8], y[8];
-        rc.get(i, f);
+        cur.get(i, f);
         if (LN) ln_chunk(f, mu, rstd, gamma_f, beta_f, c, y);
         else div_chunk(f, s, c, y);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(y[e]));
+        for (int e = 0; e < 8; ++e) {
+          amax = fmaxf(amax, fabsf(y[e]));
+          if (KEEP_Y) yk[i * 8 + e] = y[e];
+        }
       }
     }
     amax = block_max(amax, red + 2 * (ROW_WARPS + 1));
     const float scale = __fdiv_rn(amax, 127.0f);
+    const SharedDivisor d(scale);
     if (threadIdx.x == 0) sx[m] = scale;
     int8_t* qrow = xq + m * (int64_t)K;
 #pragma unroll
     for (int i = 0; i < MAXC; ++i) {
       const int c = threadIdx.x + i * ROW_THREADS;
       if (c < nchunks) {
-        float f[8], y[8];
-        rc.get(i, f);
-        if (LN) ln_chunk(f, mu, rstd, gamma_f, beta_f, c, y);
-        else div_chunk(f, s, c, y);
-        uint2 packed;
-        packed.x = pack4_s8(quant_code(y[0], scale), quant_code(y[1], scale), quant_code(y[2], scale),
-                            quant_code(y[3], scale));
-        packed.y = pack4_s8(quant_code(y[4], scale), quant_code(y[5], scale), quant_code(y[6], scale),
-                            quant_code(y[7], scale));
+        float y[8];
+        if (KEEP_Y) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = yk[i * 8 + e];
+        } else {
+          float f[8];
+          cur.get(i, f);
+          if (LN) ln_chunk(f, mu, rstd, gamma_f, beta_f, c, y);
+          else div_chunk(f, s, c, y);
+        }
+        uint2 packed = make_uint2(0u, 0u);
+        if (scale != 0.0f) {
+          packed.x = pack4_low_bytes(code_bits(y[0], d), code_bits(y[1], d), code_bits(y[2], d), code_bits(y[3], d));
+          packed.y = pack4_low_bytes(code_bits(y[4], d), code_bits(y[5], d), code_bits(y[6], d), code_bits(y[7], d));
+        }
+        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = packed;
+      }
+    }
+    if (PREFETCH) cur = nxt;
+    else if (mn < M) cur.load(x + mn * ld_bytes, nchunks);
+  }
+}
+
+// Rows of up to 16384 elements: one group of T threads per row (256 / T rows per block),
+// the row as floats in registers, the next row's raw vectors loaded as soon as the
+// current row is converted; y overwrites x in place.
+template <bool BF16, int T, int NCH, bool LN>
+__global__ void __launch_bounds__(256)
+ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
+                      const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
+                      const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx) {
+  constexpr int G = 256 / T;
+  __shared__ float red[G][24];  // per group: mean partials, variance partials, max
+  const int gid = threadIdx.x / T, t = threadIdx.x % T;
+  const int nchunks = K / 8;
+  RowRaw<BF16, NCH> raw;
+  const int64_t mstep = (int64_t)gridDim.x * G;
+  int64_t m = (int64_t)blockIdx.x * G + gid;
+  if (m < M) raw.template load<T>(x + m * ld_bytes, nchunks, t);
+  for (; m < M; m += mstep) {
+    float v[NCH * 8];
+    raw.to_float(v);
+    const int64_t mn = m + mstep;
+    if (mn < M) raw.template load<T>(x + mn * ld_bytes, nchunks, t);
+    float mu = 0.0f, rstd = 0.0f;
+    if (LN) group_row_stats<T, NCH>(v, nchunks, K, eps, red[gid], t, gid, mu, rstd);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = t + T * i;
+      if (c < nchunks) {
+        if (LN) {
+          ln_chunk(v + i * 8, mu, rstd, gamma_f, beta_f, c, v + i * 8);
+        } else {
+          div_chunk(v + i * 8, s, c, v + i * 8);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i * 8 + e]));
+      }
+    }
+    amax = group_max<T>(amax, red[gid] + 16, t, gid);
+    const float scale = __fdiv_rn(amax, 127.0f);
+    if (t == 0) sx[m] = scale;
+    const SharedDivisor d(scale);
+    int8_t* qrow = xq + m * (int64_t)K;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = t + T * i;
+      if (c < nchunks) {
+        uint2 packed = make_uint2(0u, 0u);
+        if (scale != 0.0f) {
+          const float* y = v + i * 8;
+          packed.x = pack4_low_bytes(code_bits(y[0], d), code_bits(y[1], d), code_bits(y[2], d), code_bits(y[3], d));
+          packed.y = pack4_low_bytes(code_bits(y[4], d), code_bits(y[5], d), code_bits(y[6], d), code_bits(y[7], d));
+        }
         *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = packed;
       }
     }
@@ -68,24 +146,95 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
 
 namespace sqh {
 
+template <bool BF16, int T, int NCH, bool LN>
+static cudaError_t launch_group_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
+                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
+                                  cudaStream_t st) {
+  auto kern = sqk::ln_quant_group_kernel<BF16, T, NCH, LN>;
+  int per_sm = 1;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+  if (e != cudaSuccess) return e;
+  constexpr int G = 256 / T;
+  const int64_t blocks = (M + G - 1) / G;
+  const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
+  kern<<<(unsigned)grid, 256, 0, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx);
+  return cudaGetLastError();
+}
+
+template <bool BF16, int T>
+static cudaError_t launch_group_nch(int nch, const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
+                                    const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
+                                    cudaStream_t st) {
+#define SQ_GRP(NCH)                                                                                          \
+  if (nch <= NCH)                                                                                            \
+    return gamma_f ? launch_group_t<BF16, T, NCH, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st) \
+                   : launch_group_t<BF16, T, NCH, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st);
+  SQ_GRP(1) SQ_GRP(2) SQ_GRP(4) SQ_GRP(8)
+#undef SQ_GRP
+  return cudaErrorInvalidValue;
+}
+
+// Threads per row for the group kernels: the smallest T whose chunks per thread fit in
+// `max_nch`; 0 when even T = 256 does not.
+int pick_row_threads(int64_t K, int max_nch, int* nch) {
+  const int64_t nchunks = K / 8;
+  for (int T : {32, 64, 128, 256}) {
+    const int64_t n = (nchunks + T - 1) / T;
+    if (n <= max_nch) {
+      *nch = (int)n;
+      return T;
+    }
+  }
+  return 0;
+}
+
+template <bool BF16, int MAXC, bool LN>
+static cudaError_t launch_lnq_mode(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
+                                   const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
+                                   cudaStream_t st) {
+  constexpr bool PF = BF16 && MAXC <= 4;      // register double buffer while it stays small
+  constexpr bool KEEP = MAXC <= 8;            // y in registers (64 floats at most)
+  auto kern = sqk::ln_smooth_quant_kernel<BF16, MAXC, LN, PF, KEEP>;
+  int per_sm = 1;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sqk::ROW_THREADS, 0);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(M, (int64_t)num_sms() * std::max(per_sm, 1));
+  kern<<<(unsigned)grid, sqk::ROW_THREADS, 0, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq,
+                                                    sx);
+  return cudaGetLastError();
+}
+
 template <bool BF16, int MAXC>
 static cudaError_t launch_lnq_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                 const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                 cudaStream_t st) {
-  const int64_t grid = std::min<int64_t>(M, (int64_t)num_sms() * 64);
-  if (gamma_f)
-    sqk::ln_smooth_quant_kernel<BF16, MAXC, true><<<(unsigned)grid, sqk::ROW_THREADS, 0, st>>>(
-        (const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx);
-  else
-    sqk::ln_smooth_quant_kernel<BF16, MAXC, false><<<(unsigned)grid, sqk::ROW_THREADS, 0, st>>>(
-        (const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx);
-  return cudaGetLastError();
+  if (gamma_f) return launch_lnq_mode<BF16, MAXC, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st);
+  return launch_lnq_mode<BF16, MAXC, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st);
 }
+
+bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch);
+cudaError_t launch_rowpipe_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
+                                 const float* beta_f, const float* s, float eps, int8_t* xq, float* sx, int T, int nch,
+                                 cudaStream_t st);
 
 cudaError_t launch_ln_smooth_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
                                    const float* gamma_f, const float* beta_f, const float* s, float eps,
                                    int8_t* xq, float* sx, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
+  int pT = 0, pn = 0;
+  if (K <= 8192 && rowpipe_shape(K, bf16, 8, &pT, &pn))  // staged rows win up to 8192; beyond, register prefetch
+    return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, st);
+  int nch = 0;
+  const int T = pick_row_threads(K, 8, &nch);
+  if (T) {
+    const int k = (int)K;
+#define SQ_T(TT)                                                                                      \
+  if (T == TT)                                                                                        \
+    return bf16 ? launch_group_nch<true, TT>(nch, x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, st)  \
+                : launch_group_nch<false, TT>(nch, x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, st);
+    SQ_T(32) SQ_T(64) SQ_T(128) SQ_T(256)
+#undef SQ_T
+  }
   const int need = (int)((K / 8 + sqk::ROW_THREADS - 1) / sqk::ROW_THREADS);
   const int k = (int)K;
 #define SQ_LNQ_CASE(C)                                                                                  \

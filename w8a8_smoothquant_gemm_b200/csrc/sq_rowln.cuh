@@ -149,4 +149,152 @@ __device__ __forceinline__ void div_chunk(const float x[8], const float* s, int 
   for (int e = 0; e < 8; ++e) y[e] = __fdiv_rn(x[e], sv[e]);
 }
 
+// ============================================================================ row groups
+// A row handled by a group of T threads (T in {32, 64, 128, 256}, 256 / T groups per block
+// of 256 threads).  Thread t of the group owns chunks c = t + T m (m < NCH) and, for the
+// fixed reduction order above, the 256 / T lanes t + T i: chunk c is lane c mod 256, i.e.
+// partial i = m mod (256 / T), and each partial takes its chunks in increasing m.  The row
+// is held as NCH * 8 floats in registers.
+
+template <int T>
+__device__ __forceinline__ void group_barrier(int gid) {
+  if (T == 32) {
+    __syncwarp();
+  } else if (T == 256) {
+    __syncthreads();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(gid + 1), "r"(T) : "memory");
+  }
+}
+
+// Fixed-order sum of the 256 lane partials p[0 .. 256/T) of this group; every thread of
+// the group gets the total.  `red`: 8 floats of shared memory owned by this call site.
+template <int T>
+__device__ __forceinline__ float group_sum_fixed(const float* p, float* red, int t, int gid) {
+  constexpr int P = 256 / T;
+  const int lane = t & 31, w = t >> 5;
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    float x = p[i];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x = __fadd_rn(x, __shfl_down_sync(0xffffffffu, x, o));
+    if (lane == 0) red[(T / 32) * i + w] = x;  // 32-lane group (T i + 32 w) / 32
+  }
+  group_barrier<T>(gid);
+  float g[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) g[i] = red[i];
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1)
+#pragma unroll
+    for (int i = 0; i < o; ++i) g[i] = __fadd_rn(g[i], g[i + o]);
+  return g[0];
+}
+
+// Max over the group (order-free); every thread of the group gets it.  `red`: T/32 floats.
+template <int T>
+__device__ __forceinline__ float group_max(float v, float* red, int t, int gid) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (T == 32) return v;
+  if ((t & 31) == 0) red[t >> 5] = v;
+  group_barrier<T>(gid);
+  float m = red[0];
+#pragma unroll
+  for (int i = 1; i < T / 32; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+// Raw 16-byte vectors of the chunks a thread owns (for loads ahead of use).
+template <bool BF16, int NCH>
+struct RowRaw {
+  static constexpr int VEC = BF16 ? 1 : 2;
+  uint4 v[NCH * VEC];
+  template <int T>
+  __device__ __forceinline__ void load(const char* row, int nchunks, int t) {
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+      const int c = t + T * m;
+      if (c < nchunks) {
+#pragma unroll
+        for (int h = 0; h < VEC; ++h) v[m * VEC + h] = ldg_stream16(row + (size_t)c * 16 * VEC + 16 * h);
+      }
+    }
+  }
+  __device__ __forceinline__ void to_float(float* f) const {
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+      if (BF16) {
+        unpack8_bf16(v[m], f + m * 8);
+      } else {
+        const uint4 a = v[m * VEC], b = v[m * VEC + VEC - 1];
+        f[m * 8 + 0] = __uint_as_float(a.x); f[m * 8 + 1] = __uint_as_float(a.y);
+        f[m * 8 + 2] = __uint_as_float(a.z); f[m * 8 + 3] = __uint_as_float(a.w);
+        f[m * 8 + 4] = __uint_as_float(b.x); f[m * 8 + 5] = __uint_as_float(b.y);
+        f[m * 8 + 6] = __uint_as_float(b.z); f[m * 8 + 7] = __uint_as_float(b.w);
+      }
+    }
+  }
+};
+
+// mu and rstd of the row v[] (chunks c = t + T m) in the fixed order.  red: 16 floats.
+template <int T, int NCH>
+__device__ __forceinline__ void group_row_stats(const float* v, int nchunks, int K, float eps, float* red, int t,
+                                                int gid, float& mu, float& rstd) {
+  constexpr int P = 256 / T;
+  float p[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) p[i] = 0.0f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m)
+    if (t + T * m < nchunks)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) p[m % P] = __fadd_rn(p[m % P], v[m * 8 + e]);
+  const float kf = (float)K;
+  mu = __fdiv_rn(group_sum_fixed<T>(p, red, t, gid), kf);
+#pragma unroll
+  for (int i = 0; i < P; ++i) p[i] = 0.0f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m)
+    if (t + T * m < nchunks)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = __fsub_rn(v[m * 8 + e], mu);
+        p[m % P] = __fmaf_rn(d, d, p[m % P]);
+      }
+  const float var = __fdiv_rn(group_sum_fixed<T>(p, red + 8, t, gid), kf);
+  rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
+}
+
+// As group_row_stats, but leaves d = x - mu in v[] (the LayerNorm output is then
+// fma(d * rstd, gamma, beta)) and returns only rstd.
+template <int T, int NCH>
+__device__ __forceinline__ void group_row_stats_d(float* v, int nchunks, int K, float eps, float* red, int t, int gid,
+                                                  float& rstd) {
+  constexpr int P = 256 / T;
+  float p[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) p[i] = 0.0f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m)
+    if (t + T * m < nchunks)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) p[m % P] = __fadd_rn(p[m % P], v[m * 8 + e]);
+  const float kf = (float)K;
+  const float mu = __fdiv_rn(group_sum_fixed<T>(p, red, t, gid), kf);
+#pragma unroll
+  for (int i = 0; i < P; ++i) p[i] = 0.0f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m)
+    if (t + T * m < nchunks)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = __fsub_rn(v[m * 8 + e], mu);
+        v[m * 8 + e] = d;
+        p[m % P] = __fmaf_rn(d, d, p[m % P]);
+      }
+  const float var = __fdiv_rn(group_sum_fixed<T>(p, red + 8, t, gid), kf);
+  rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
+}
+
 }  // namespace sqk

@@ -1,0 +1,290 @@
+// sq_rowpipe.cu -- activation-row kernels with TMA bulk-copy staging:
+//   LN_QUANT     fused LayerNorm (folded gamma' = gamma/s, beta' = beta/s) -> per-token INT8
+//   PLAIN_QUANT  y = x / s (input from a previous GEMM)                     -> per-token INT8
+//   LN_CALIB     per-channel absmax of LayerNorm(x) with the original gamma, beta
+// ("4.2 W8A8 量化与 SmoothQuant", sec. 6 and 7.1; "量化：只压权重，与训练后量化（PTQ）",
+// per-token activation quantisation.)
+//
+// A block of 256 threads holds 256 / T row groups of T threads.  Each group's first thread
+// streams whole rows (cp.async.bulk, K * elt bytes) into the group's S-slot ring in shared
+// memory, S rows ahead, completing on one mbarrier per slot; the per-channel vectors
+// (gamma', beta' -- or s and RN(1/s) -- or gamma, beta) are copied to shared memory once per
+// block.  A slot is refilled as soon as every thread of the group has moved its row into
+// registers, which the row's first group barrier guarantees.  Row statistics use the fixed
+// reduction order of sq_rowln.cuh; codes use the shared-divisor quantiser of sq_common.cuh.
+#include <algorithm>
+
+#include "sq_ptx.cuh"
+#include "sq_rowln.cuh"
+
+namespace sqk {
+
+enum RowMode : int { ROW_LN_QUANT = 0, ROW_PLAIN_QUANT = 1, ROW_LN_CALIB = 2 };
+
+template <bool BF16, int T, int NCH, int S, int MODE>
+__global__ void __launch_bounds__(256)
+rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, const float* __restrict__ vec_a,
+               const float* __restrict__ vec_b, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
+               float* __restrict__ out, unsigned int* err) {
+  constexpr int G = 256 / T;
+  constexpr int ELT = BF16 ? 2 : 4;
+  constexpr bool LN = MODE != ROW_PLAIN_QUANT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  float* sa = reinterpret_cast<float*>(sm);  // gamma' | s | gamma      [K]
+  float* sb = sa + K;                          // beta'  | 1/s | beta     [K]
+  const int row_bytes = K * ELT;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(sb + K);  // [G][S][row_bytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)G * S * row_bytes);  // [G][S]
+  __shared__ float red[G][24];
+
+  const int gid = threadIdx.x / T, t = threadIdx.x % T;
+  const int nchunks = K / 8;
+
+  // per-channel vectors, once per block
+  int slow = 0;
+  for (int j = threadIdx.x; j < K; j += 256) {
+    const float a = vec_a[j];
+    sa[j] = a;
+    if (MODE == ROW_PLAIN_QUANT) {
+      const bool fast = fabsf(a) >= 0x1p-90f && fabsf(a) <= 0x1p+90f;
+      slow |= !fast;
+      sb[j] = fast ? __frcp_rn(a) : 0.0f;
+    } else {
+      sb[j] = vec_b ? vec_b[j] : 0.0f;
+    }
+  }
+  if (t == 0) {
+    for (int k = 0; k < S; ++k) mbar_init(smem_u32(&bars[gid * S + k]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const bool all_fast = !__syncthreads_or(slow);
+
+  uint8_t* gring = ring + (size_t)gid * S * row_bytes;
+  const int64_t rstep = (int64_t)gridDim.x * G;
+  const int64_t r0 = (int64_t)blockIdx.x * G + gid;
+  auto issue = [&](int slot, int64_t r) {
+    const uint32_t b = smem_u32(&bars[gid * S + slot]);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(b, (uint32_t)row_bytes);
+    bulk_load(smem_u32(gring + (size_t)slot * row_bytes), x + r * ld_bytes, (uint32_t)row_bytes, b);
+  };
+  if (t == 0)
+    for (int k = 0; k < S; ++k)
+      if (r0 + k * rstep < M) issue(k, r0 + k * rstep);
+
+  float cm[MODE == ROW_LN_CALIB ? NCH * 8 : 1];
+  if (MODE == ROW_LN_CALIB) {
+#pragma unroll
+    for (int i = 0; i < NCH * 8; ++i) cm[i] = 0.0f;
+  }
+
+  int64_t it = 0;
+  for (int64_t r = r0; r < M; r += rstep, ++it) {
+    const int slot = (int)(it % S);
+    if (!mbar_wait(smem_u32(&bars[gid * S + slot]), (uint32_t)((it / S) & 1))) atomicOr(err, ERR_ROW_TMA_WAIT);
+    const uint8_t* rowp = gring + (size_t)slot * row_bytes;
+    float v[NCH * 8];
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+      const int c = t + T * m;
+      if (c < nchunks) {
+        if (BF16) {
+          unpack8_bf16(*reinterpret_cast<const uint4*>(rowp + (size_t)c * 16), v + m * 8);
+        } else {
+          const uint4 a = *reinterpret_cast<const uint4*>(rowp + (size_t)c * 32);
+          const uint4 b = *reinterpret_cast<const uint4*>(rowp + (size_t)c * 32 + 16);
+          v[m * 8 + 0] = __uint_as_float(a.x); v[m * 8 + 1] = __uint_as_float(a.y);
+          v[m * 8 + 2] = __uint_as_float(a.z); v[m * 8 + 3] = __uint_as_float(a.w);
+          v[m * 8 + 4] = __uint_as_float(b.x); v[m * 8 + 5] = __uint_as_float(b.y);
+          v[m * 8 + 6] = __uint_as_float(b.z); v[m * 8 + 7] = __uint_as_float(b.w);
+        }
+      }
+    }
+    // ---- y in v[]
+    if (LN) {
+      float rstd;
+      group_row_stats_d<T, NCH>(v, nchunks, K, eps, red[gid], t, gid, rstd);  // v <- x - mu
+      if (t == 0 && r + S * rstep < M) issue(slot, r + S * rstep);           // slot drained
+#pragma unroll
+      for (int m = 0; m < NCH; ++m) {
+        const int c = t + T * m;
+        if (c < nchunks) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float4 g = *reinterpret_cast<const float4*>(sa + c * 8 + h * 4);
+            const float4 b = *reinterpret_cast<const float4*>(sb + c * 8 + h * 4);
+            float* d = v + m * 8 + h * 4;
+            d[0] = __fmaf_rn(__fmul_rn(d[0], rstd), g.x, b.x);
+            d[1] = __fmaf_rn(__fmul_rn(d[1], rstd), g.y, b.y);
+            d[2] = __fmaf_rn(__fmul_rn(d[2], rstd), g.z, b.z);
+            d[3] = __fmaf_rn(__fmul_rn(d[3], rstd), g.w, b.w);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < NCH; ++m) {
+        const int c = t + T * m;
+        if (c < nchunks) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float4 sv = *reinterpret_cast<const float4*>(sa + c * 8 + h * 4);
+            const float4 rv = *reinterpret_cast<const float4*>(sb + c * 8 + h * 4);
+            float* d = v + m * 8 + h * 4;
+            if (all_fast) {
+              // Markstein: q = RN(x y), r = x - s q exact, RN(q + r y) = RN(x / s)
+              float q;
+              q = __fmul_rn(d[0], rv.x); d[0] = __fmaf_rn(__fmaf_rn(-q, sv.x, d[0]), rv.x, q);
+              q = __fmul_rn(d[1], rv.y); d[1] = __fmaf_rn(__fmaf_rn(-q, sv.y, d[1]), rv.y, q);
+              q = __fmul_rn(d[2], rv.z); d[2] = __fmaf_rn(__fmaf_rn(-q, sv.z, d[2]), rv.z, q);
+              q = __fmul_rn(d[3], rv.w); d[3] = __fmaf_rn(__fmaf_rn(-q, sv.w, d[3]), rv.w, q);
+            } else {
+              d[0] = __fdiv_rn(d[0], sv.x);
+              d[1] = __fdiv_rn(d[1], sv.y);
+              d[2] = __fdiv_rn(d[2], sv.z);
+              d[3] = __fdiv_rn(d[3], sv.w);
+            }
+          }
+        }
+      }
+    }
+    if (MODE == ROW_LN_CALIB) {
+#pragma unroll
+      for (int m = 0; m < NCH; ++m)
+        if (t + T * m < nchunks)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) cm[m * 8 + e] = fmaxf(cm[m * 8 + e], fabsf(v[m * 8 + e]));
+      continue;
+    }
+    // ---- per-token quantisation
+    float amax = 0.0f;
+#pragma unroll
+    for (int m = 0; m < NCH; ++m)
+      if (t + T * m < nchunks)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[m * 8 + e]));
+    amax = group_max<T>(amax, red[gid] + 16, t, gid);
+    if (!LN && t == 0 && r + S * rstep < M) issue(slot, r + S * rstep);  // slot drained
+    const float scale = __fdiv_rn(amax, 127.0f);
+    if (t == 0) sx[r] = scale;
+    const SharedDivisor dv(scale);
+    int8_t* qrow = xq + r * (int64_t)K;
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+      const int c = t + T * m;
+      if (c < nchunks) {
+        const float* y = v + m * 8;
+        uint2 packed;
+        packed.x = pack4_low_bytes(code_bits(y[0], dv), code_bits(y[1], dv), code_bits(y[2], dv), code_bits(y[3], dv));
+        packed.y = pack4_low_bytes(code_bits(y[4], dv), code_bits(y[5], dv), code_bits(y[6], dv), code_bits(y[7], dv));
+        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = packed;
+      }
+    }
+  }
+
+  if (MODE == ROW_LN_CALIB) {
+    // merge the groups' column maxima through shared memory (the ring is idle now), then
+    // one atomicMax per column per block
+    __syncthreads();
+    float* scratch = reinterpret_cast<float*>(ring);  // [G][K]
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+      const int c = t + T * m;
+      if (c < nchunks)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) scratch[gid * K + c * 8 + e] = cm[m * 8 + e];
+    }
+    __syncthreads();
+    if ((int64_t)blockIdx.x * G < M)
+      for (int j = threadIdx.x; j < K; j += 256) {
+        float mx = scratch[j];
+#pragma unroll
+        for (int g = 1; g < G; ++g) mx = fmaxf(mx, scratch[g * K + j]);
+        atomic_max_nonneg(out + j, mx);
+      }
+  }
+}
+
+}  // namespace sqk
+
+namespace sqh {
+
+int pick_row_threads(int64_t K, int max_nch, int* nch);
+
+// Shared memory of one block: two per-channel vectors, the rings, the barriers.
+static size_t rowpipe_smem(int K, int elt, int G, int S) {
+  return 128 + (size_t)K * 8 + (size_t)G * S * K * elt + (size_t)G * S * 8;
+}
+
+template <bool BF16, int T, int NCH, int MODE>
+static cudaError_t launch_rowpipe_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
+                                    const float* vb, float eps, int8_t* xq, float* sx, float* out, cudaStream_t st) {
+  constexpr int G = 256 / T;
+  constexpr int S = 2;
+  auto kern = sqk::rowpipe_kernel<BF16, T, NCH, S, MODE>;
+  const size_t smem = rowpipe_smem(K, BF16 ? 2 : 4, G, S);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 1;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (M + G - 1) / G;
+  const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
+  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, va, vb, eps, xq, sx, out, error_word_ptr());
+  return cudaGetLastError();
+}
+
+template <bool BF16, int T, int MODE>
+static cudaError_t launch_rowpipe_nch(int nch, const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
+                                      const float* vb, float eps, int8_t* xq, float* sx, float* out,
+                                      cudaStream_t st) {
+  if (nch <= 1) return launch_rowpipe_t<BF16, T, 1, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+  if (nch <= 2) return launch_rowpipe_t<BF16, T, 2, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+  if (nch <= 4) return launch_rowpipe_t<BF16, T, 4, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+  // calibration keeps at most 4 chunks per thread (its running maxima live in registers too)
+  if (MODE == sqk::ROW_LN_CALIB) return cudaErrorInvalidValue;
+  constexpr int N8 = MODE == sqk::ROW_LN_CALIB ? 4 : 8;
+  return launch_rowpipe_t<BF16, T, N8, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+}
+
+template <int MODE>
+static cudaError_t launch_rowpipe_mode(bool bf16, int T, int nch, const void* x, int64_t M, int K, int64_t ld_bytes,
+                                       const float* va, const float* vb, float eps, int8_t* xq, float* sx, float* out,
+                                       cudaStream_t st) {
+#define SQ_T(TT)                                                                                          \
+  if (T == TT)                                                                                            \
+    return bf16 ? launch_rowpipe_nch<true, TT, MODE>(nch, x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st) \
+                : launch_rowpipe_nch<false, TT, MODE>(nch, x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+  SQ_T(32) SQ_T(64) SQ_T(128) SQ_T(256)
+#undef SQ_T
+  return cudaErrorInvalidValue;
+}
+
+// Whether the staged row kernel applies (rows of up to 8 chunks per thread whose block fits
+// the shared memory); sets threads per row and chunks per thread.
+bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch) {
+  *T = pick_row_threads(K, max_nch, nch);
+  if (!*T) return false;
+  return rowpipe_smem((int)K, bf16 ? 2 : 4, 256 / *T, 2) <= 200 * 1024;
+}
+
+cudaError_t launch_rowpipe_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
+                                 const float* beta_f, const float* s, float eps, int8_t* xq, float* sx, int T, int nch,
+                                 cudaStream_t st) {
+  const int64_t ldb = ldx * (bf16 ? 2 : 4);
+  if (gamma_f)
+    return launch_rowpipe_mode<sqk::ROW_LN_QUANT>(bf16, T, nch, x, M, (int)K, ldb, gamma_f, beta_f, eps, xq, sx,
+                                                  nullptr, st);
+  return launch_rowpipe_mode<sqk::ROW_PLAIN_QUANT>(bf16, T, nch, x, M, (int)K, ldb, s, nullptr, eps, xq, sx, nullptr,
+                                                   st);
+}
+
+cudaError_t launch_rowpipe_calib(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx, const float* gamma,
+                                 const float* beta, float eps, float* out, int T, int nch, cudaStream_t st) {
+  const int64_t ldb = ldx * (bf16 ? 2 : 4);
+  return launch_rowpipe_mode<sqk::ROW_LN_CALIB>(bf16, T, nch, x, rows, (int)K, ldb, gamma, beta, eps, nullptr, nullptr,
+                                                out, st);
+}
+
+}  // namespace sqh
