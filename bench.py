@@ -90,6 +90,14 @@ def max_over_ranks(v: float, world: int, device) -> float:
     return float(t.item())
 
 
+def combine_statistic(ax: torch.Tensor, world: int) -> None:
+    """Each rank calibrates on its own tokens; the absmax over the whole calibration set is the
+    element-wise max over ranks (an all-reduce, in place).  A no-op on one rank."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(ax, op=dist.ReduceOp.MAX)
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples of one GPU while the timed region runs."""
@@ -162,9 +170,7 @@ class Linear:
             sq.sq_calib_ln_absmax(self.x, self.gamma, out=self.ax)
         else:
             sq.sq_calib_absmax(self.x, 0, out=self.ax)
-        if world > 1:
-            import torch.distributed as dist
-            dist.all_reduce(self.ax, op=dist.ReduceOp.MAX)
+        combine_statistic(self.ax, world)
         sq.sq_calib_absmax(self.W, 1, out=self.aw)
         sq.sq_smooth_factors(self.ax, self.aw, ALPHA, out=self.s)
         sq.sq_fold_quant_weights(self.W, self.s, self.gamma if self.ln else None, wq=self.wq, sw=self.sw,
