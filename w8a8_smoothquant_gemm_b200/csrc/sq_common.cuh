@@ -64,6 +64,10 @@ struct SharedDivisor {
   }
   __device__ __forceinline__ float div(float a) const {
     if (!fast) return __fdiv_rn(a, b);
+    return div_fast(a);
+  }
+  // Markstein quotient only; valid when `fast` (callers branch once, outside their loops).
+  __device__ __forceinline__ float div_fast(float a) const {
     const float q = __fmul_rn(a, y);
     const float r = __fmaf_rn(-q, b, a);
     return __fmaf_rn(r, y, q);
@@ -79,10 +83,22 @@ struct SharedDivisor {
 __device__ __forceinline__ uint32_t code_bits(float v, const SharedDivisor& d) {
   return __float_as_uint(__fadd_rn(d.div(v), 12582912.0f));
 }
+__device__ __forceinline__ uint32_t code_bits_fast(float v, const SharedDivisor& d) {
+  return __float_as_uint(__fadd_rn(d.div_fast(v), 12582912.0f));
+}
 
 // Low bytes of four words -> one packed word (first argument in the low byte).
 __device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Codes of 8 values (one chunk) packed into 8 bytes; FAST selects the Markstein-only path.
+template <bool FAST>
+__device__ __forceinline__ uint2 pack8_codes(const float* y, const SharedDivisor& d) {
+  uint32_t c[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) c[e] = FAST ? code_bits_fast(y[e], d) : code_bits(y[e], d);
+  return make_uint2(pack4_low_bytes(c[0], c[1], c[2], c[3]), pack4_low_bytes(c[4], c[5], c[6], c[7]));
 }
 
 // Packs four codes (low byte first) into one 32-bit word.

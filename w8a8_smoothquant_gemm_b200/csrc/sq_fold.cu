@@ -159,11 +159,47 @@ fold_quant_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_
 // ---------------------------------------------------------------------------- cluster fold
 // One thread-block cluster of C CTAs per strip of CW output channels.  CTA r of the
 // cluster owns rows [r * RK, (r + 1) * RK) of W (input channels): one thread TMA-loads that
-// RK x CW block into shared memory (W crosses HBM once), the CTA reduces its partial
-// column maxima of |s_j W_jk|, the C partials are combined through distributed shared
-// memory, and the CTA quantises its block from shared memory, writing Wq[k, j] transposed
-// (each thread emits 64 consecutive j of one k).  Rows beyond K and columns beyond N are
-// zero-filled by TMA and never stored.
+// RK x CW block into shared memory in 64-row pieces, each completing on its own mbarrier,
+// so the column-max pass follows the data in (W crosses HBM once).  Each CTA pushes its
+// partial column maxima of |s_j W_jk| into every peer's shared memory (distributed shared
+// memory), one cluster barrier later every CTA has all C partials, and it quantises its
+// block from shared memory, writing Wq[k, j] transposed, 16 codes at a time.  Rows beyond
+// K and columns beyond N are zero-filled by TMA and never stored.
+// Codes of a 16-row x 4-column block of the staged tile (rows jl.., columns kq..kq+3),
+// as 4 words per column; FAST selects the Markstein-only division.
+template <bool FAST>
+__device__ __forceinline__ void fold_codes_16x4(const uint16_t* tile, const float* s_rows, int cw, int jl, int kq,
+                                                const SharedDivisor& d0, const SharedDivisor& d1,
+                                                const SharedDivisor& d2, const SharedDivisor& d3,
+                                                uint32_t (&words)[4][4]) {
+#pragma unroll
+  for (int g4 = 0; g4 < 4; ++g4) {
+    uint32_t b[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = jl + g4 * 4 + r;
+      const uint2 w = *reinterpret_cast<const uint2*>(tile + j * cw + kq);
+      const float sj = s_rows[j];
+      if (FAST) {
+        b[0][r] = code_bits_fast(__fmul_rn(sj, bf16lo(w.x)), d0);
+        b[1][r] = code_bits_fast(__fmul_rn(sj, bf16hi(w.x)), d1);
+        b[2][r] = code_bits_fast(__fmul_rn(sj, bf16lo(w.y)), d2);
+        b[3][r] = code_bits_fast(__fmul_rn(sj, bf16hi(w.y)), d3);
+      } else {
+        b[0][r] = code_bits(__fmul_rn(sj, bf16lo(w.x)), d0);
+        b[1][r] = code_bits(__fmul_rn(sj, bf16hi(w.x)), d1);
+        b[2][r] = code_bits(__fmul_rn(sj, bf16lo(w.y)), d2);
+        b[3][r] = code_bits(__fmul_rn(sj, bf16hi(w.y)), d3);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) words[c][g4] = pack4_low_bytes(b[c][0], b[c][1], b[c][2], b[c][3]);
+  }
+}
+
+constexpr int FOLD_MAX_CLUSTER = 16;
+constexpr int FOLD_MAX_PIECES = 64;  // RK <= 4096 rows per CTA
+
 template <int CW>
 __global__ void __launch_bounds__(256)
 fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t N, int RK, int C,
@@ -177,15 +213,16 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
   const uint16_t* tile = reinterpret_cast<const uint16_t*>(smem);      // [RK][CW] bf16 bits
   float* s_rows = reinterpret_cast<float*>(smem + (size_t)RK * CW * 2);  // [RK]
   __shared__ float red[G][CW + 1];
-  __shared__ float part[CW];
+  __shared__ float part[FOLD_MAX_CLUSTER][CW];  // partial maxima of every CTA of the cluster
   __shared__ float scale[CW];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bars[FOLD_MAX_PIECES];
 
   const int tid = threadIdx.x;
   const uint32_t crank = cluster_ctarank();
   const int64_t strip = blockIdx.x / C;
   const int64_t k0 = strip * CW;
   const int64_t j0 = (int64_t)crank * RK;
+  const int pieces = RK / 64;
 
   for (int64_t j = (int64_t)blockIdx.x * 256 + tid; j < K; j += (int64_t)gridDim.x * 256) {
     const float sj = s[j];
@@ -193,34 +230,39 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
     if (beta && beta_f) beta_f[j] = __fdiv_rn(beta[j], sj);
   }
 
-  const uint32_t b = smem_u32(&bar);
   if (tid == 0) {
-    mbar_init(b, 1);
+    for (int p = 0; p < pieces; ++p) mbar_init(smem_u32(&bars[p]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncthreads();
   if (tid == 0) {
-    mbar_arrive_expect_tx(b, (uint32_t)RK * CW * 2);
-    for (int r = 0; r < RK; r += 64) tma_load_2d(smem_u32(smem + (size_t)r * CW * 2), &wmap, b, (int)k0, (int)(j0 + r));
+    for (int p = 0; p < pieces; ++p) {
+      const uint32_t b = smem_u32(&bars[p]);
+      mbar_arrive_expect_tx(b, (uint32_t)64 * CW * 2);
+      tma_load_2d(smem_u32(smem + (size_t)p * 64 * CW * 2), &wmap, b, (int)k0, (int)(j0 + p * 64));
+    }
   }
   for (int i = tid; i < RK; i += 256) s_rows[i] = (j0 + i < K) ? __ldg(s + j0 + i) : 0.0f;
-  if (!mbar_wait(b, 0)) atomicOr(err, ERR_FOLD_TMA_WAIT);
   __syncthreads();
 
-  // ---- partial column max of |s_j W_jk| over this CTA's rows: thread = 8 columns x rows rl + G m
+  // ---- partial column max of |s_j W_jk| over this CTA's rows, piece by piece as they land:
+  // thread = 8 columns x rows rl, rl + G, ...
   {
     const int cg = tid % (CW / 8), rl = tid / (CW / 8);
     float m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = 0.0f;
-    for (int j = rl; j < RK; j += G) {
-      const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
-      const float sj = s_rows[j];
-      float f[8];
-      unpack8_bf16(w, f);
+    for (int p = 0; p < pieces; ++p) {
+      if (!mbar_wait(smem_u32(&bars[p]), 0)) atomicOr(err, ERR_FOLD_TMA_WAIT);
+      for (int j = p * 64 + rl; j < p * 64 + 64; j += G) {
+        const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
+        const float sj = s_rows[j];
+        float f[8];
+        unpack8_bf16(w, f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(sj, f[e])));
+        for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(sj, f[e])));
+      }
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
@@ -229,12 +271,12 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
   if (tid < CW) {
     float m = red[0][tid];
     for (int g = 1; g < G; ++g) m = fmaxf(m, red[g][tid]);
-    part[tid] = m;
+    for (int r = 0; r < C; ++r) st_dsmem_f32(&part[crank][tid], (uint32_t)r, m);  // into every CTA
   }
-  cluster_sync();
+  cluster_sync();  // all partials delivered; no CTA touches a peer's memory after this
   if (tid < CW) {
     float m = 0.0f;
-    for (int r = 0; r < C; ++r) m = fmaxf(m, ld_dsmem_f32(&part[tid], (uint32_t)r));
+    for (int r = 0; r < C; ++r) m = fmaxf(m, part[r][tid]);
     const float sc = __fdiv_rn(m, 127.0f);
     scale[tid] = sc;
     if (crank == 0 && k0 + tid < N) sw[k0 + tid] = sc;
@@ -249,22 +291,10 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
     if (j0 + jl >= K) continue;  // K % 16 == 0: a 16-row block is all in or all out
     const SharedDivisor d0(scale[kq]), d1(scale[kq + 1]), d2(scale[kq + 2]), d3(scale[kq + 3]);
     uint32_t words[4][4];
-#pragma unroll
-    for (int g4 = 0; g4 < 4; ++g4) {
-      uint32_t b[4][4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j = jl + g4 * 4 + r;
-        const uint2 w = *reinterpret_cast<const uint2*>(tile + j * CW + kq);
-        const float sj = s_rows[j];
-        b[0][r] = code_bits(__fmul_rn(sj, bf16lo(w.x)), d0);
-        b[1][r] = code_bits(__fmul_rn(sj, bf16hi(w.x)), d1);
-        b[2][r] = code_bits(__fmul_rn(sj, bf16lo(w.y)), d2);
-        b[3][r] = code_bits(__fmul_rn(sj, bf16hi(w.y)), d3);
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) words[c][g4] = pack4_low_bytes(b[c][0], b[c][1], b[c][2], b[c][3]);
-    }
+    if (d0.fast && d1.fast && d2.fast && d3.fast)
+      fold_codes_16x4<true>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
+    else
+      fold_codes_16x4<false>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int64_t k = k0 + kq + c;
@@ -272,7 +302,6 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
         *reinterpret_cast<uint4*>(Wq + k * K + j0 + jl) = make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
     }
   }
-  cluster_sync();  // peers may still be reading `part` through distributed shared memory
 }
 
 }  // namespace sqk
@@ -337,18 +366,19 @@ static cudaError_t launch_fold_cluster_t(const void* W, int64_t K, int64_t N, in
   return cudaLaunchKernelEx(&cfg, kern, map, K, N, RK, C, s, gamma, beta, Wq, sw, gamma_f, beta_f, error_word_ptr());
 }
 
-// Cluster shape of the single-pass fold: the widest strip (CW) and smallest cluster (C)
-// whose per-CTA block fits `budget` bytes of shared memory.
+// Cluster shape of the single-pass fold: C CTAs share a strip (at least 256 rows each, at
+// most 16), and the strip is the widest CW whose per-CTA block fits `budget` bytes of
+// shared memory.
 static bool fold_cluster_shape(int64_t K, size_t budget, int* cw, int* c, int* rk) {
+  const int cl = (int)std::min<int64_t>(16, std::max<int64_t>(1, (K + 255) / 256));
+  const int64_t rows = ((K + cl - 1) / cl + 63) / 64 * 64;
+  if (rows / 64 > sqk::FOLD_MAX_PIECES) return false;
   for (int w : {64, 32, 16})
-    for (int cl : {1, 2, 4, 8, 16}) {
-      const int64_t rows = ((K + cl - 1) / cl + 63) / 64 * 64;
-      if ((size_t)rows * w * 2 + (size_t)rows * 4 <= budget) {
-        *cw = w;
-        *c = cl;
-        *rk = (int)rows;
-        return true;
-      }
+    if ((size_t)rows * w * 2 + (size_t)rows * 4 <= budget) {
+      *cw = w;
+      *c = cl;
+      *rk = (int)rows;
+      return true;
     }
   return false;
 }

@@ -46,7 +46,9 @@ struct GemmParams {
   int num_kb;                // ceil(K / BK)
   int kb_per_split, splits;
   int num_units;             // tiles_a * tiles_b * splits
-  int group_a;               // raster: this many A tiles share a sweep over B tiles
+  int group_a;               // raster (b_major = 0): this many A tiles share a sweep over B tiles
+  int group_b;               // raster (b_major = 1): this many B tiles share a sweep over A tiles
+  int b_major;
   int M, N;                  // output is y[M, N]
   const float* sx;
   const float* sw;
@@ -175,17 +177,29 @@ __device__ __forceinline__ void store_out(const GemmParams& p, int64_t m, int64_
 }
 
 // Unit u -> (A tile, B tile, K split).  Splits of one tile are adjacent so they run
-// concurrently; tiles are rastered in groups of group_a A tiles for L2 reuse.
+// concurrently.  Tiles are rastered so that one operand stays resident in L2 while the
+// other streams through once: a group of group_a A tiles sweeps over all B tiles (A tile
+// index fastest), or, with b_major, a group of group_b B tiles sweeps over all A tiles.
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta, int& tb, int& split) {
   split = u % p.splits;
   const int tile = u / p.splits;
-  const int group_size = p.group_a * p.tiles_b;
-  const int group = tile / group_size;
-  const int first_a = group * p.group_a;
-  const int ga = min(p.tiles_a - first_a, p.group_a);
-  const int in_group = tile % group_size;
-  ta = first_a + in_group % ga;
-  tb = in_group / ga;
+  if (!p.b_major) {
+    const int group_size = p.group_a * p.tiles_b;
+    const int group = tile / group_size;
+    const int first_a = group * p.group_a;
+    const int ga = min(p.tiles_a - first_a, p.group_a);
+    const int in_group = tile % group_size;
+    ta = first_a + in_group % ga;
+    tb = in_group / ga;
+  } else {
+    const int group_size = p.group_b * p.tiles_a;
+    const int group = tile / group_size;
+    const int first_b = group * p.group_b;
+    const int gb = min(p.tiles_b - first_b, p.group_b);
+    const int in_group = tile % group_size;
+    tb = first_b + in_group % gb;
+    ta = in_group / gb;
+  }
 }
 
 // Shared-memory layout of one CTA: BN_CTA rows of B per stage (BN / CG), BN accumulator
@@ -616,7 +630,22 @@ cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, con
   p.kb_per_split = pl.kb_per_split;
   p.splits = pl.splits;
   p.num_units = pl.tiles_a * pl.tiles_b * pl.splits;
-  p.group_a = pl.swap ? 1 : 16 / pl.cg;
+  // Keep the smaller operand resident in L2 (up to ~48 MB of it per group) and stream the
+  // larger one through once.
+  {
+    const int64_t tile_m = (int64_t)sqk::BM * pl.cg, tile_n = pl.swap ? pl.bn : 256;
+    const int64_t a_bytes = (pl.swap ? N : M) * K, b_bytes = (pl.swap ? M : N) * K;
+    const int64_t budget = 48ll << 20;
+    if (a_bytes <= b_bytes) {
+      p.b_major = 0;
+      p.group_a = (int)std::max<int64_t>(1, std::min<int64_t>(pl.tiles_a, budget / std::max<int64_t>(1, tile_m * K)));
+      p.group_b = 1;
+    } else {
+      p.b_major = 1;
+      p.group_b = (int)std::max<int64_t>(1, std::min<int64_t>(pl.tiles_b, budget / std::max<int64_t>(1, tile_n * K)));
+      p.group_a = 1;
+    }
+  }
   p.M = (int)M;
   p.N = (int)N;
   p.sx = sx;

@@ -94,8 +94,20 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
                       const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx) {
   constexpr int G = 256 / T;
   __shared__ float red[G][24];  // per group: mean partials, variance partials, max
+  extern __shared__ float rs[];  // plain mode: RN(1 / s_j), or 0 where s_j is outside the fast range
   const int gid = threadIdx.x / T, t = threadIdx.x % T;
   const int nchunks = K / 8;
+  bool all_fast = true;
+  if (!LN) {
+    int slow = 0;
+    for (int j = threadIdx.x; j < K; j += 256) {
+      const float a = s[j];
+      const bool fast = fabsf(a) >= 0x1p-90f && fabsf(a) <= 0x1p+90f;
+      slow |= !fast;
+      rs[j] = fast ? __frcp_rn(a) : 0.0f;
+    }
+    all_fast = !__syncthreads_or(slow);
+  }
   RowRaw<BF16, NCH> raw;
   const int64_t mstep = (int64_t)gridDim.x * G;
   int64_t m = (int64_t)blockIdx.x * G + gid;
@@ -107,36 +119,50 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
     if (mn < M) raw.template load<T>(x + mn * ld_bytes, nchunks, t);
     float mu = 0.0f, rstd = 0.0f;
     if (LN) group_row_stats<T, NCH>(v, nchunks, K, eps, red[gid], t, gid, mu, rstd);
-    float amax = 0.0f;
+    float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent max chains
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = t + T * i;
       if (c < nchunks) {
         if (LN) {
           ln_chunk(v + i * 8, mu, rstd, gamma_f, beta_f, c, v + i * 8);
+        } else if (all_fast) {
+          // y = x / s_j through the shared divisor s_j with y_j = RN(1/s_j) (Markstein)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float4 sv = __ldg(reinterpret_cast<const float4*>(s + (size_t)c * 8 + h * 4));
+            const float4 rv = *reinterpret_cast<const float4*>(rs + c * 8 + h * 4);
+            float* d = v + i * 8 + h * 4;
+            float q;
+            q = __fmul_rn(d[0], rv.x); d[0] = __fmaf_rn(__fmaf_rn(-q, sv.x, d[0]), rv.x, q);
+            q = __fmul_rn(d[1], rv.y); d[1] = __fmaf_rn(__fmaf_rn(-q, sv.y, d[1]), rv.y, q);
+            q = __fmul_rn(d[2], rv.z); d[2] = __fmaf_rn(__fmaf_rn(-q, sv.z, d[2]), rv.z, q);
+            q = __fmul_rn(d[3], rv.w); d[3] = __fmaf_rn(__fmaf_rn(-q, sv.w, d[3]), rv.w, q);
+          }
         } else {
           div_chunk(v + i * 8, s, c, v + i * 8);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i * 8 + e]));
+        for (int e = 0; e < 8; ++e) am[e] = fmaxf(am[e], fabsf(v[i * 8 + e]));
       }
     }
+    float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
     amax = group_max<T>(amax, red[gid] + 16, t, gid);
     const float scale = __fdiv_rn(amax, 127.0f);
     if (t == 0) sx[m] = scale;
     const SharedDivisor d(scale);
     int8_t* qrow = xq + m * (int64_t)K;
+    if (d.fast) {
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int c = t + T * i;
-      if (c < nchunks) {
-        uint2 packed = make_uint2(0u, 0u);
-        if (scale != 0.0f) {
-          const float* y = v + i * 8;
-          packed.x = pack4_low_bytes(code_bits(y[0], d), code_bits(y[1], d), code_bits(y[2], d), code_bits(y[3], d));
-          packed.y = pack4_low_bytes(code_bits(y[4], d), code_bits(y[5], d), code_bits(y[6], d), code_bits(y[7], d));
-        }
-        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = packed;
+      for (int i = 0; i < NCH; ++i) {
+        const int c = t + T * i;
+        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<true>(v + i * 8, d);
+      }
+    } else {  // rare: a scale outside the fast range
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int c = t + T * i;
+        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false>(v + i * 8, d);
       }
     }
   }
@@ -151,13 +177,16 @@ static cudaError_t launch_group_t(const void* x, int64_t M, int K, int64_t ld_by
                                   const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                   cudaStream_t st) {
   auto kern = sqk::ln_quant_group_kernel<BF16, T, NCH, LN>;
+  const size_t smem = LN ? 0 : sizeof(float) * (size_t)K;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   int per_sm = 1;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
   if (e != cudaSuccess) return e;
   constexpr int G = 256 / T;
   const int64_t blocks = (M + G - 1) / G;
   const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
-  kern<<<(unsigned)grid, 256, 0, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx);
+  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx);
   return cudaGetLastError();
 }
 
@@ -222,7 +251,7 @@ cudaError_t launch_ln_smooth_quant(const void* x, bool bf16, int64_t M, int64_t 
                                    int8_t* xq, float* sx, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   int pT = 0, pn = 0;
-  if (K <= 8192 && rowpipe_shape(K, bf16, 8, &pT, &pn))  // staged rows win up to 8192; beyond, register prefetch
+  if (K <= 8192 && rowpipe_shape(K, bf16, 4, &pT, &pn))  // staged rows, 4 chunks per thread  // staged rows win up to 8192; beyond, register prefetch
     return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, st);
   int nch = 0;
   const int T = pick_row_threads(K, 8, &nch);

@@ -158,27 +158,30 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
       continue;
     }
     // ---- per-token quantisation
-    float amax = 0.0f;
+    float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent max chains
 #pragma unroll
     for (int m = 0; m < NCH; ++m)
       if (t + T * m < nchunks)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[m * 8 + e]));
+        for (int e = 0; e < 8; ++e) am[e] = fmaxf(am[e], fabsf(v[m * 8 + e]));
+    float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
     amax = group_max<T>(amax, red[gid] + 16, t, gid);
     if (!LN && t == 0 && r + S * rstep < M) issue(slot, r + S * rstep);  // slot drained
     const float scale = __fdiv_rn(amax, 127.0f);
     if (t == 0) sx[r] = scale;
     const SharedDivisor dv(scale);
     int8_t* qrow = xq + r * (int64_t)K;
+    if (dv.fast) {
 #pragma unroll
-    for (int m = 0; m < NCH; ++m) {
-      const int c = t + T * m;
-      if (c < nchunks) {
-        const float* y = v + m * 8;
-        uint2 packed;
-        packed.x = pack4_low_bytes(code_bits(y[0], dv), code_bits(y[1], dv), code_bits(y[2], dv), code_bits(y[3], dv));
-        packed.y = pack4_low_bytes(code_bits(y[4], dv), code_bits(y[5], dv), code_bits(y[6], dv), code_bits(y[7], dv));
-        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = packed;
+      for (int m = 0; m < NCH; ++m) {
+        const int c = t + T * m;
+        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<true>(v + m * 8, dv);
+      }
+    } else {  // rare: a scale outside the fast range
+#pragma unroll
+      for (int m = 0; m < NCH; ++m) {
+        const int c = t + T * m;
+        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false>(v + m * 8, dv);
       }
     }
   }
