@@ -123,6 +123,43 @@ absmax_rows_kernel(const char* __restrict__ x, int64_t rows, int64_t nvec, int64
   if (threadIdx.x == 0) out[r] = accumulate ? fmaxf(out[r], m) : m;
 }
 
+// Short rows (up to 8 KB): one warp per row, every 16-byte vector of the row loaded at once
+// (up to 16 per lane in flight), shuffle reduction, no block barrier.
+template <bool BF16, int VPL>
+__global__ void __launch_bounds__(256)
+absmax_rows_warp_kernel(const char* __restrict__ x, int64_t rows, int64_t nvec, int64_t ld_bytes, int accumulate,
+                        float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const char* p = x + r * ld_bytes;
+  uint4 q[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if (lane + 32 * i < nvec) q[i] = ldg_stream16(p + (int64_t)(lane + 32 * i) * 16);
+  float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    if (lane + 32 * i < nvec) {
+      if (BF16) {
+        float f[8];
+        unpack8_bf16(q[i], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e & 3] = fmaxf(m[e & 3], fabsf(f[e]));
+      } else {
+        m[0] = fmaxf(m[0], fabsf(__uint_as_float(q[i].x)));
+        m[1] = fmaxf(m[1], fabsf(__uint_as_float(q[i].y)));
+        m[2] = fmaxf(m[2], fabsf(__uint_as_float(q[i].z)));
+        m[3] = fmaxf(m[3], fabsf(__uint_as_float(q[i].w)));
+      }
+    }
+  }
+  float v = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) out[r] = accumulate ? fmaxf(out[r], v) : v;
+}
+
 // ---------------------------------------------------------------------------- LayerNorm output
 // Blocks loop over rows; each thread keeps the running max of the elements of its own
 // chunks -- in registers (REG, rows of up to 32 elements per thread) or in shared memory --
@@ -257,6 +294,18 @@ cudaError_t launch_absmax(const void* x, bool bf16, int64_t rows, int64_t cols, 
       sqk::absmax_cols_kernel<true><<<grid, block, 0, st>>>((const char*)x, rows, nvec, ld_bytes, out);
     else
       sqk::absmax_cols_kernel<false><<<grid, block, 0, st>>>((const char*)x, rows, nvec, ld_bytes, out);
+  } else if (nvec <= 32 * 16) {  // rows up to 8 KB: a warp per row
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+#define SQ_RW(V)                                                                                                   \
+  if (nvec <= 32 * V) {                                                                                            \
+    if (bf16)                                                                                                      \
+      sqk::absmax_rows_warp_kernel<true, V><<<grid, 256, 0, st>>>((const char*)x, rows, nvec, ld_bytes, accumulate, out); \
+    else                                                                                                           \
+      sqk::absmax_rows_warp_kernel<false, V><<<grid, 256, 0, st>>>((const char*)x, rows, nvec, ld_bytes, accumulate, out); \
+    return cudaGetLastError();                                                                                     \
+  }
+    SQ_RW(2) SQ_RW(4) SQ_RW(8) SQ_RW(16)
+#undef SQ_RW
   } else {
     if (bf16)
       sqk::absmax_rows_kernel<true><<<(unsigned)rows, 256, 0, st>>>((const char*)x, rows, nvec, ld_bytes, accumulate, out);

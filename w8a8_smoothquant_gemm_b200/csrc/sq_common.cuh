@@ -92,12 +92,28 @@ __device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Codes of 8 values (one chunk) packed into 8 bytes; FAST selects the Markstein-only path.
+// Codes of 8 values (one chunk) packed into 8 bytes; FAST selects the Markstein-only path,
+// evaluated two lanes at a time with packed binary32 arithmetic (each half rounds exactly
+// as the scalar operation would).
 template <bool FAST>
 __device__ __forceinline__ uint2 pack8_codes(const float* y, const SharedDivisor& d) {
   uint32_t c[8];
+  if (FAST) {
+    const float2 rc = make_float2(d.y, d.y), nb = make_float2(-d.b, -d.b);
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) c[e] = FAST ? code_bits_fast(y[e], d) : code_bits(y[e], d);
+    for (int e = 0; e < 8; e += 2) {
+      const float2 a = make_float2(y[e], y[e + 1]);
+      const float2 q = __fmul2_rn(a, rc);
+      const float2 r = __ffma2_rn(q, nb, a);
+      const float2 t = __fadd2_rn(__ffma2_rn(r, rc, q), magic);
+      c[e] = __float_as_uint(t.x);
+      c[e + 1] = __float_as_uint(t.y);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c[e] = code_bits(y[e], d);
+  }
   return make_uint2(pack4_low_bytes(c[0], c[1], c[2], c[3]), pack4_low_bytes(c[4], c[5], c[6], c[7]));
 }
 

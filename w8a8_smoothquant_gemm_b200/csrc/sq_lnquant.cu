@@ -88,7 +88,7 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
 // the row as floats in registers, the next row's raw vectors loaded as soon as the
 // current row is converted; y overwrites x in place.
 template <bool BF16, int T, int NCH, bool LN>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
                       const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
                       const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx) {
@@ -104,7 +104,7 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
       const float a = s[j];
       const bool fast = fabsf(a) >= 0x1p-90f && fabsf(a) <= 0x1p+90f;
       slow |= !fast;
-      rs[j] = fast ? __frcp_rn(a) : 0.0f;
+      rs[(((j & 7) >> 2) * nchunks + (j >> 3)) * 4 + (j & 3)] = fast ? __frcp_rn(a) : 0.0f;  // [half][chunk]
     }
     all_fast = !__syncthreads_or(slow);
   }
@@ -131,7 +131,7 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const float4 sv = __ldg(reinterpret_cast<const float4*>(s + (size_t)c * 8 + h * 4));
-            const float4 rv = *reinterpret_cast<const float4*>(rs + c * 8 + h * 4);
+            const float4 rv = *reinterpret_cast<const float4*>(rs + (h * nchunks + c) * 4);
             float* d = v + i * 8 + h * 4;
             float q;
             q = __fmul_rn(d[0], rv.x); d[0] = __fmaf_rn(__fmaf_rn(-q, sv.x, d[0]), rv.x, q);

@@ -41,17 +41,20 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
   const int gid = threadIdx.x / T, t = threadIdx.x % T;
   const int nchunks = K / 8;
 
-  // per-channel vectors, once per block
+  // per-channel vectors, once per block, as float4s ordered [half][chunk] (element j sits at
+  // ((j % 8) / 4 * nchunks + j / 8) * 4 + j % 4) so that a thread's read of its chunk's half
+  // h is 16 bytes after its neighbour's: conflict-free.
   int slow = 0;
   for (int j = threadIdx.x; j < K; j += 256) {
+    const int at = (((j & 7) >> 2) * nchunks + (j >> 3)) * 4 + (j & 3);
     const float a = vec_a[j];
-    sa[j] = a;
+    sa[at] = a;
     if (MODE == ROW_PLAIN_QUANT) {
       const bool fast = fabsf(a) >= 0x1p-90f && fabsf(a) <= 0x1p+90f;
       slow |= !fast;
-      sb[j] = fast ? __frcp_rn(a) : 0.0f;
+      sb[at] = fast ? __frcp_rn(a) : 0.0f;
     } else {
-      sb[j] = vec_b ? vec_b[j] : 0.0f;
+      sb[at] = vec_b ? vec_b[j] : 0.0f;
     }
   }
   if (t == 0) {
@@ -112,13 +115,15 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
         if (c < nchunks) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const float4 g = *reinterpret_cast<const float4*>(sa + c * 8 + h * 4);
-            const float4 b = *reinterpret_cast<const float4*>(sb + c * 8 + h * 4);
+            const float4 g = *reinterpret_cast<const float4*>(sa + (h * nchunks + c) * 4);
+            const float4 b = *reinterpret_cast<const float4*>(sb + (h * nchunks + c) * 4);
             float* d = v + m * 8 + h * 4;
-            d[0] = __fmaf_rn(__fmul_rn(d[0], rstd), g.x, b.x);
-            d[1] = __fmaf_rn(__fmul_rn(d[1], rstd), g.y, b.y);
-            d[2] = __fmaf_rn(__fmul_rn(d[2], rstd), g.z, b.z);
-            d[3] = __fmaf_rn(__fmul_rn(d[3], rstd), g.w, b.w);
+            const float2 rs2 = make_float2(rstd, rstd);
+            const float2 y01 = __ffma2_rn(__fmul2_rn(make_float2(d[0], d[1]), rs2), make_float2(g.x, g.y),
+                                          make_float2(b.x, b.y));
+            const float2 y23 = __ffma2_rn(__fmul2_rn(make_float2(d[2], d[3]), rs2), make_float2(g.z, g.w),
+                                          make_float2(b.z, b.w));
+            d[0] = y01.x; d[1] = y01.y; d[2] = y23.x; d[3] = y23.y;
           }
         }
       }
@@ -129,16 +134,18 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
         if (c < nchunks) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const float4 sv = *reinterpret_cast<const float4*>(sa + c * 8 + h * 4);
-            const float4 rv = *reinterpret_cast<const float4*>(sb + c * 8 + h * 4);
+            const float4 sv = *reinterpret_cast<const float4*>(sa + (h * nchunks + c) * 4);
+            const float4 rv = *reinterpret_cast<const float4*>(sb + (h * nchunks + c) * 4);
             float* d = v + m * 8 + h * 4;
             if (all_fast) {
-              // Markstein: q = RN(x y), r = x - s q exact, RN(q + r y) = RN(x / s)
-              float q;
-              q = __fmul_rn(d[0], rv.x); d[0] = __fmaf_rn(__fmaf_rn(-q, sv.x, d[0]), rv.x, q);
-              q = __fmul_rn(d[1], rv.y); d[1] = __fmaf_rn(__fmaf_rn(-q, sv.y, d[1]), rv.y, q);
-              q = __fmul_rn(d[2], rv.z); d[2] = __fmaf_rn(__fmaf_rn(-q, sv.z, d[2]), rv.z, q);
-              q = __fmul_rn(d[3], rv.w); d[3] = __fmaf_rn(__fmaf_rn(-q, sv.w, d[3]), rv.w, q);
+              // Markstein: q = RN(x y), r = x - s q exact, RN(q + r y) = RN(x / s), two lanes at a time
+              const float2 x01 = make_float2(d[0], d[1]), x23 = make_float2(d[2], d[3]);
+              const float2 r01 = make_float2(rv.x, rv.y), r23 = make_float2(rv.z, rv.w);
+              const float2 q01 = __fmul2_rn(x01, r01), q23 = __fmul2_rn(x23, r23);
+              const float2 e01 = __ffma2_rn(q01, make_float2(-sv.x, -sv.y), x01);
+              const float2 e23 = __ffma2_rn(q23, make_float2(-sv.z, -sv.w), x23);
+              const float2 y01 = __ffma2_rn(e01, r01, q01), y23 = __ffma2_rn(e23, r23, q23);
+              d[0] = y01.x; d[1] = y01.y; d[2] = y23.x; d[3] = y23.y;
             } else {
               d[0] = __fdiv_rn(d[0], sv.x);
               d[1] = __fdiv_rn(d[1], sv.y);
