@@ -44,6 +44,30 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 INT8_PER_BF16 = 2.0  # dense INT8 tensor rate / dense BF16 rate on B200 (4.5 vs 2.25 PFLOP/s nominal)
 
 
+def gemm_traffic() -> int | None:
+    """DRAM bytes per GEMM launch of this step from the committed ncu summary, or None when the
+    GEMM sources changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "w8a8_gemm_pair_prefill8b_traffic.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.split(":")[0].strip().isidentifier():
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "w8a8_smoothquant_gemm_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("sq_gemm.cu", "sq_ptx.cuh"):
+        h.update(open(os.path.join(src, f), "rb").read())
+    if fields.get("gemm_source_sha256_16") != h.hexdigest()[:16]:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def step_ops(M: int = TOKENS) -> float:
     return float(sum(2.0 * M * N * K for _, K, N, _ in LAYERS))
 
@@ -360,7 +384,9 @@ def run_device(args, rank, world, local):
     gemm_ops = [2.0 * L.M * L.N * L.K for L in layers]
     achieved = sum(gemm_ops) / sum(gemm_s) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": int8_peak, "unit": "TOPS",
-                "frac": round(achieved / int8_peak, 4), "traffic": None,
+                "frac": round(achieved / int8_peak, 4), "traffic": gemm_traffic(),
+                "traffic_unit": "DRAM bytes per GEMM launch (mean of the 4 launches of a step)",
+                "algorithmic_bytes_per_launch": int(sum(L.M * L.K + L.N * L.K + 2 * L.M * L.N for L in layers) / 4),
                 "kernel": "w8a8_gemm_kernel (tcgen05 kind::i8), 4 launches per step",
                 "peak_note": f"2 x {peaks['source']} burst bf16 {peaks['bf16_tflops']} TFLOP/s"}
     per_gemm = {L.name: {"us": round(t * 1e6, 1), "tops": round(o / t / 1e12, 1),
