@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
         L.sqo_calib_ln_absmax.restype = None
         L.sqo_ln_smooth_quant.argtypes = [P, I, I64, I64, I64, P, P, P, F, P, P]
         L.sqo_ln_smooth_quant.restype = None
+        L.sqo_ln_smooth_quant_per_tensor.argtypes = [P, I, I64, I64, I64, P, P, P, F, I, P, P, P]
+        L.sqo_ln_smooth_quant_per_tensor.restype = None
         L.sqo_quant_per_tensor.argtypes = [P, I64, P, P]
         L.sqo_quant_per_tensor.restype = None
         L.sqo_w8a8_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I, I64]
@@ -171,6 +173,23 @@ def ln_smooth_quant(x: np.ndarray, gamma_f=None, beta_f=None, s=None, eps: float
                               _ptr(_c(beta_f, np.float32)), _ptr(_c(s, np.float32)), float(eps),
                               _ptr(xq), _ptr(sx))
     return xq, sx
+
+
+def ln_smooth_quant_per_tensor(x: np.ndarray, gamma_f=None, beta_f=None, s=None, eps: float = 1e-5,
+                               static_scale: float | None = None):
+    """One scale for the whole tensor: max|y|/127 (dynamic) or the given calibrated scale
+    (static, values beyond it clamp to +-127).  Returns (xq, sx [every row = scale], scale)."""
+    if (gamma_f is None) == (s is None):
+        raise ValueError("exactly one of gamma_f (LayerNorm mode) and s (plain mode) is given")
+    x = _c(x)
+    M, K = x.shape
+    xq = np.empty((M, K), np.int8)
+    sx = np.empty(M, np.float32)
+    sc = np.array([0.0 if static_scale is None else static_scale], np.float32)
+    lib().sqo_ln_smooth_quant_per_tensor(_ptr(x), _dtype_code(x), M, K, K, _ptr(_c(gamma_f, np.float32)),
+                                         _ptr(_c(beta_f, np.float32)), _ptr(_c(s, np.float32)), float(eps),
+                                         int(static_scale is not None), _ptr(sc), _ptr(xq), _ptr(sx))
+    return xq, sx, float(sc[0])
 
 
 def quant_per_tensor(y: np.ndarray):

@@ -310,6 +310,47 @@ void sqo_ln_smooth_quant(const void* x, int dt, int64_t M, int64_t K, int64_t ld
 }
 
 /* ---------------------------------------------------------------------------
+ * Fused LayerNorm / smoothing -> per-TENSOR INT8 (the coarser activation granularity:
+ * one scale for the whole activation tensor)  [SQ-pipe] (O1 and the static end of the
+ * granularity ladder), [Q8]
+ *   y as in sqo_ln_smooth_quant;
+ *   static_scale == 0: scale = max_{m,j} |y_mj| / 127 (dynamic), written to *scale;
+ *   static_scale != 0: scale = *scale as given (calibrated); values beyond it clamp.
+ *   xq_mj = clamp(rne(y_mj / scale), -127, 127);  sx[m] = scale for every row.
+ * ------------------------------------------------------------------------- */
+void sqo_ln_smooth_quant_per_tensor(const void* x, int dt, int64_t M, int64_t K, int64_t ldx,
+                                    const float* gamma_f, const float* beta_f, const float* s,
+                                    float eps, int static_scale, float* scale, int8_t* xq,
+                                    float* sx) {
+  float* y = (float*)malloc(sizeof(float) * (size_t)(M * K > 0 ? M * K : 1));
+  float* xr = (float*)malloc(sizeof(float) * (size_t)K);
+  float* tmp = (float*)malloc(sizeof(float) * (size_t)K);
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t j = 0; j < K; ++j) xr[j] = load_elt(x, dt, m * ldx + j);
+    if (gamma_f) {
+      layernorm_row(xr, K, gamma_f, beta_f, eps, y + m * K, tmp);
+    } else {
+      for (int64_t j = 0; j < K; ++j) y[m * K + j] = xr[j] / s[j];
+    }
+  }
+  float sc;
+  if (static_scale) {
+    sc = *scale;
+  } else {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < M * K; ++i) {
+      const float a = fabsf(y[i]);
+      if (a > amax) amax = a;
+    }
+    sc = amax / 127.0f;
+    *scale = sc;
+  }
+  for (int64_t i = 0; i < M * K; ++i) xq[i] = quant_code(y[i], sc);
+  for (int64_t m = 0; m < M; ++m) sx[m] = sc;
+  free(y); free(xr); free(tmp);
+}
+
+/* ---------------------------------------------------------------------------
  * Per-tensor symmetric INT8 (the coarse activation granularity the pages compare
  * against):  scale = max |y| / 127 over the whole tensor  [Q8], [SQ-pipe]
  * ------------------------------------------------------------------------- */

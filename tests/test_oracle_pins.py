@@ -345,3 +345,52 @@ def test_pipeline_error_bound_tiny_case():
         assert np.all(np.abs(Yh - Y) <= bound * (1 + 1e-4) + 1e-6)
         errs[alpha] = _rel_fro(Yh, Y)
     assert errs[0.5] < errs[None]
+
+
+# ----------------------------------------------------------------------------- per-tensor granularity
+def test_per_tensor_dynamic_matches_the_demo_rule_on_the_whole_tensor():
+    """Per-tensor: the demo's quantize_int8 (one max/127 for the whole matrix) applied to y."""
+    rng = np.random.default_rng(30)
+    x = rng.standard_normal((7, 64)).astype(np.float32)
+    x[:, 9] *= 80
+    s = rng.uniform(0.5, 4.0, 64).astype(np.float32)
+    xq, sx, scale = O.ln_smooth_quant_per_tensor(x, s=s)
+    y = x / s[None, :]
+    ref_scale = np.float32(np.max(np.abs(y))) / np.float32(127.0)
+    assert scale == ref_scale and np.all(sx == ref_scale)
+    assert np.array_equal(xq, np.clip(np.round(y / ref_scale), -127, 127).astype(np.int8))
+    q2, s2 = O.quant_per_tensor(y)
+    assert np.array_equal(q2, xq) and s2 == scale
+
+
+def test_per_tensor_is_coarser_than_per_token():
+    """The PTQ page's ladder: per-token activations quantise the outlier example more finely
+    than one per-tensor scale (1.76% vs 1.95% without smoothing)."""
+    g = json.load(open(os.path.join(GOLDEN, "p4_worked_example.json")))
+    X = np.array(g["X"], np.float32)
+    W = np.array(g["W"], np.float32)
+    wq, sw, _, _ = O.fold_quant_weights(W, np.ones(3, np.float32))
+    Y = X.astype(np.float64) @ W.astype(np.float64)
+    qt, sxt, _ = O.ln_smooth_quant_per_tensor(X, s=np.ones(3, np.float32))
+    qk, sxk = O.ln_smooth_quant(X, s=np.ones(3, np.float32))
+    e_tensor = _rel_fro(O.dequant_linear_f64(qt, sxt, wq, sw), Y)
+    e_token = _rel_fro(O.dequant_linear_f64(qk, sxk, wq, sw), Y)
+    assert abs(e_tensor - g["rel_err_per_tensor_act"][0]) <= g["rel_err_per_tensor_abs"][0]
+    assert e_token < e_tensor
+
+
+def test_per_tensor_static_scale_clamps():
+    """A calibrated scale smaller than this batch's max: codes saturate at +-127, the rest round."""
+    x = np.array([[0.5, -300.0, 2.5, 1000.0, -1.5, 3.5, 0.0, 127.0]], np.float32)
+    xq, sx, scale = O.ln_smooth_quant_per_tensor(x, s=np.ones(8, np.float32), static_scale=1.0)
+    assert scale == 1.0 and sx.tolist() == [1.0]
+    assert xq.tolist() == [[0, -127, 2, 127, -2, 4, 0, 127]]
+
+
+def test_per_tensor_layernorm_mode_uses_the_same_layernorm():
+    c = sq_inputs.make_case(6, 256, 8, 31, beta_std=0.1)
+    y = O.layernorm(c.x, c.gamma, c.beta)
+    xq, sx, scale = O.ln_smooth_quant_per_tensor(c.x, gamma_f=c.gamma, beta_f=c.beta)
+    assert scale == np.float32(np.max(np.abs(y))) / np.float32(127.0)
+    q2, _ = O.quant_per_tensor(y)
+    assert np.array_equal(xq, q2)
