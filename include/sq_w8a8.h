@@ -117,6 +117,20 @@ sq_status sq_ln_smooth_quant(const void* x, sq_dtype dt, int64_t M, int64_t K, i
                              const float* gamma_f, const float* beta_f, const float* s, float eps,
                              int8_t* xq, float* sx, void* stream);
 
+/* sq_ln_smooth_quant_per_tensor -- the same y as sq_ln_smooth_quant, quantised with ONE scale
+ * for the whole activation tensor (the coarser per-tensor granularity of "4.2 W8A8…" sec. 7.1
+ * and of "量化…PTQ": static per-tensor at the coarse end, dynamic per-token at the fine end):
+ *   static_scale = 0 (dynamic): scale = max_{m,j} |y[m, j]| / 127, written to *scale;
+ *   static_scale = 1 (static, calibrated): *scale is read (positive, finite);
+ *   xq[m, j] = clamp(rne(y[m, j] / scale), -127, 127) -- values beyond a static scale saturate;
+ *   sx[m] = scale for every row, so sq_w8a8_gemm applies it unchanged.
+ *   scale: one fp32 in device memory.  Other arguments as for sq_ln_smooth_quant.  The
+ *   dynamic form makes two passes over x (statistics, then codes) and uses sx as scratch
+ *   in between. */
+sq_status sq_ln_smooth_quant_per_tensor(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                        const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                        int static_scale, float* scale, int8_t* xq, float* sx, void* stream);
+
 /* sq_w8a8_gemm -- INT8 x INT8 -> int32 GEMM on the tcgen05 tensor cores with the dequant
  * epilogue ("4.2 W8A8…" intro: the GEMM runs on INT8 tensor cores; "量化…PTQ": per-token
  * and per-channel scales are multiplied back after the GEMM):

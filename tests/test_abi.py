@@ -154,3 +154,24 @@ def test_workspace_size_validation():
 
 def test_device_error_null_pointer():
     assert sq.lib().sq_device_error(NULL, 0, NULL) == INVALID
+
+
+def test_ln_smooth_quant_per_tensor_validation():
+    f = sq.lib().sq_ln_smooth_quant_per_tensor
+    ok = (A16, BF16, 4, 64, 64, NULL, NULL, A16c, 1e-5, 0, A16b, A16c, A16b, NULL)
+    args = list(ok)
+    args[10] = NULL
+    assert f(*args) == INVALID                       # no scale
+    args = list(ok)
+    args[9] = 2
+    assert f(*args) == INVALID                       # static flag not 0/1
+    args = list(ok)
+    args[5] = A16b
+    assert f(*args) == INVALID                       # both modes
+    args = list(ok)
+    args[3] = 40
+    args[4] = 40
+    assert f(*args) == ALIGN                         # K % 16
+    args = list(ok)
+    args[2] = 0
+    assert f(*args) == 0                             # M = 0: nothing to do

@@ -310,3 +310,54 @@ def test_large_layer_sampled_rows(M, K, N, ln, w_std):
     assert np.array_equal(g["xq"][rows], xq) and np.array_equal(g["sx"][rows], sx)
     ref = O.w8a8_gemm(xq, sx, g["wq"], g["sw"], "bf16")
     assert assert_bf16_close(g["y"][rows], ref) == 1.0
+
+
+# ----------------------------------------------------------------------------- per-tensor granularity
+@pytest.mark.parametrize("M,K", [(1, 16), (33, 256), (64, 4096), (9, 14336), (2, 49152), (300, 1040)])
+@pytest.mark.parametrize("mode", ["ln", "plain"])
+def test_per_tensor_dynamic(M, K, mode):
+    c = sq_inputs.make_case(M, K, 8, 5 * M + K, beta_std=0.05)
+    rng = np.random.default_rng(K + 2)
+    s = np.exp(rng.uniform(-1, 3, K)).astype(np.float32)
+    if mode == "ln":
+        gf, bf = (c.gamma / s).astype(np.float32), (c.beta / s).astype(np.float32)
+        xq, sx, sc = sq.sq_ln_smooth_quant_per_tensor(dev(c.x), gamma_f=dev(gf), beta_f=dev(bf))
+        r_xq, r_sx, r_sc = O.ln_smooth_quant_per_tensor(c.x, gamma_f=gf, beta_f=bf)
+    else:
+        xq, sx, sc = sq.sq_ln_smooth_quant_per_tensor(dev(c.x), s=dev(s))
+        r_xq, r_sx, r_sc = O.ln_smooth_quant_per_tensor(c.x, s=s)
+    assert host(sc)[0] == np.float32(r_sc)
+    assert np.array_equal(host(sx), r_sx)
+    assert np.array_equal(host(xq), r_xq)
+
+
+@pytest.mark.parametrize("K", [256, 4096, 14336, 49152])
+@pytest.mark.parametrize("mode", ["ln", "plain"])
+def test_per_tensor_static_clamps(K, mode):
+    """A calibrated scale at half the batch's own: the largest values saturate at +-127."""
+    M = 40
+    c = sq_inputs.make_case(M, K, 8, K + 9)
+    s = np.ones(K, np.float32)
+    kw = dict(gamma_f=c.gamma) if mode == "ln" else dict(s=s)
+    _, _, dyn = O.ln_smooth_quant_per_tensor(c.x, **kw)
+    static = np.float32(dyn * 0.5)
+    r_xq, r_sx, _ = O.ln_smooth_quant_per_tensor(c.x, static_scale=float(static), **kw)
+    dkw = {k: dev(v) for k, v in kw.items()}
+    xq, sx, sc = sq.sq_ln_smooth_quant_per_tensor(dev(c.x), scale=dev(np.array([static], np.float32)), static=True,
+                                                  **dkw)
+    assert np.array_equal(host(sx), r_sx) and host(sc)[0] == static
+    assert np.array_equal(host(xq), r_xq)
+    assert (np.abs(r_xq) == 127).sum() > 0
+
+
+def test_per_tensor_linear_end_to_end():
+    """Per-tensor activations through the GEMM: sx holds the one scale for every row."""
+    c = sq_inputs.make_case(48, 512, 384, 77)
+    W, x, g = dev(c.W), dev(c.x), dev(c.gamma)
+    s = sq.sq_smooth_factors(sq.sq_calib_ln_absmax(x, g), sq.sq_calib_absmax(W, 1), 0.5)
+    wq, sw, gf, _ = sq.sq_fold_quant_weights(W, s, g)
+    xq, sx, _ = sq.sq_ln_smooth_quant_per_tensor(x, gamma_f=gf)
+    y = sq.sq_w8a8_gemm(xq, sx, wq, sw)
+    r_xq, r_sx, _ = O.ln_smooth_quant_per_tensor(c.x, gamma_f=host(gf))
+    assert np.array_equal(host(xq), r_xq)
+    assert assert_bf16_close(host(y), O.w8a8_gemm(r_xq, r_sx, host(wq), host(sw), "bf16")) == 1.0

@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
             "sq_smooth_factors": [P, P, I64, F, P, P],
             "sq_fold_quant_weights": [P, I, I64, I64, I64, P, P, P, P, P, P, P, P],
             "sq_ln_smooth_quant": [P, I, I64, I64, I64, P, P, P, F, P, P, P],
+            "sq_ln_smooth_quant_per_tensor": [P, I, I64, I64, I64, P, P, P, F, I, P, P, P, P],
             "sq_w8a8_gemm": [P, P, P, P, I64, I64, I64, P, I, I64, P, SZ, P],
             "sq_device_error": [P, I, P],
         }
@@ -193,6 +194,33 @@ def sq_ln_smooth_quant(x: torch.Tensor, gamma_f: torch.Tensor | None = None, bet
                                                           _ptr(beta_f), _ptr(s), float(eps), _ptr(xq), _ptr(sx),
                                                           _stream(stream)))
     return xq, sx
+
+
+def sq_ln_smooth_quant_per_tensor(x: torch.Tensor, gamma_f: torch.Tensor | None = None,
+                                  beta_f: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                                  eps: float = 1e-5, scale: torch.Tensor | None = None, static: bool = False,
+                                  xq: torch.Tensor | None = None, sx: torch.Tensor | None = None, stream=None):
+    """One scale for the whole tensor: dynamic (max|y|/127, written to `scale`) or static (the
+    calibrated value in `scale`).  Returns (xq [M, K] int8, sx [M] = scale, scale [1])."""
+    x = _mat(x, "x")
+    M, K = x.shape
+    _vec(gamma_f, K, "gamma_f")
+    _vec(beta_f, K, "beta_f")
+    _vec(s, K, "s")
+    if scale is None:
+        if static:
+            raise ValueError("a static per-tensor scale must be given")
+        scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    _vec(scale, 1, "scale")
+    if xq is None:
+        xq = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check("sq_ln_smooth_quant_per_tensor",
+           lib().sq_ln_smooth_quant_per_tensor(_ptr(x), _dt(x), M, K, x.stride(0), _ptr(gamma_f), _ptr(beta_f),
+                                               _ptr(s), float(eps), int(static), _ptr(scale), _ptr(xq), _ptr(sx),
+                                               _stream(stream)))
+    return xq, sx, scale
 
 
 def sq_w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:

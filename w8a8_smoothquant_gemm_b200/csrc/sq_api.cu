@@ -19,6 +19,10 @@ cudaError_t launch_fold_quant(const void* W, bool bf16, int64_t K, int64_t N, in
 cudaError_t launch_ln_smooth_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                                    const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                    cudaStream_t st);
+cudaError_t launch_ln_smooth_quant_per_tensor(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
+                                              const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                              int static_scale, float* scale, int8_t* xq, float* sx,
+                                              cudaStream_t st);
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
                         int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
                         bool* ws_too_small);
@@ -160,6 +164,28 @@ sq_status sq_ln_smooth_quant(const void* x, sq_dtype dt, int64_t M, int64_t K, i
   if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
   return cuda_status(
       sqh::launch_ln_smooth_quant(x, dt == SQ_BF16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, as_stream(stream)));
+}
+
+sq_status sq_ln_smooth_quant_per_tensor(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                        const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                        int static_scale, float* scale, int8_t* xq, float* sx, void* stream) {
+  if (static_scale != 0 && static_scale != 1) return SQ_ERR_INVALID_ARG;
+  if (scale == nullptr || !aligned4(scale)) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  if ((gamma_f == nullptr) == (s == nullptr)) return SQ_ERR_INVALID_ARG;  // exactly one mode
+  if (gamma_f == nullptr && beta_f != nullptr) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_matrix(x, dt, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if ((gamma_f && !aligned16(gamma_f)) || (beta_f && !aligned16(beta_f)) || (s && !aligned16(s)))
+    return SQ_ERR_ALIGNMENT;
+  if (gamma_f && !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;
+  if (xq == nullptr || sx == nullptr || !aligned4(sx)) return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || !aligned16(xq)) return SQ_ERR_ALIGNMENT;
+  if (K > SQ_MAX_K_ROW || (dt == SQ_F32 && K > SQ_MAX_K_ROW / 2)) return SQ_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  return cuda_status(sqh::launch_ln_smooth_quant_per_tensor(x, dt == SQ_BF16, M, K, ldx, gamma_f, beta_f, s, eps,
+                                                            static_scale, scale, xq, sx, as_stream(stream)));
 }
 
 size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {

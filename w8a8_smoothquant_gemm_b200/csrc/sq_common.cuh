@@ -94,8 +94,9 @@ __device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint
 
 // Codes of 8 values (one chunk) packed into 8 bytes; FAST selects the Markstein-only path,
 // evaluated two lanes at a time with packed binary32 arithmetic (each half rounds exactly
-// as the scalar operation would).
-template <bool FAST>
+// as the scalar operation would).  CLAMP bounds the quotient to [-127, 127] first, which a
+// scale that did not come from this data's own absmax (a calibrated per-tensor scale) needs.
+template <bool FAST, bool CLAMP = false>
 __device__ __forceinline__ uint2 pack8_codes(const float* y, const SharedDivisor& d) {
   uint32_t c[8];
   if (FAST) {
@@ -106,15 +107,43 @@ __device__ __forceinline__ uint2 pack8_codes(const float* y, const SharedDivisor
       const float2 a = make_float2(y[e], y[e + 1]);
       const float2 q = __fmul2_rn(a, rc);
       const float2 r = __ffma2_rn(q, nb, a);
-      const float2 t = __fadd2_rn(__ffma2_rn(r, rc, q), magic);
+      float2 qq = __ffma2_rn(r, rc, q);
+      if (CLAMP) qq = make_float2(fminf(fmaxf(qq.x, -127.0f), 127.0f), fminf(fmaxf(qq.y, -127.0f), 127.0f));
+      const float2 t = __fadd2_rn(qq, magic);
       c[e] = __float_as_uint(t.x);
       c[e + 1] = __float_as_uint(t.y);
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) c[e] = code_bits(y[e], d);
+    for (int e = 0; e < 8; ++e) {
+      float q = d.div(y[e]);
+      if (CLAMP) q = fminf(fmaxf(q, -127.0f), 127.0f);
+      c[e] = __float_as_uint(__fadd_rn(q, 12582912.0f));
+    }
   }
   return make_uint2(pack4_low_bytes(c[0], c[1], c[2], c[3]), pack4_low_bytes(c[4], c[5], c[6], c[7]));
+}
+
+// Writes the codes of NCH chunks (chunk m of this thread at c = t + T m) of one row.
+template <int T, int NCH>
+__device__ __forceinline__ void store_row_codes(const float* v, int t, int nchunks, float scale, bool clamp,
+                                                int8_t* qrow) {
+  const SharedDivisor d(scale);
+  if (d.fast && !clamp) {
+#pragma unroll
+    for (int m = 0; m < NCH; ++m)
+      if (t + T * m < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)(t + T * m) * 8) = pack8_codes<true>(v + m * 8, d);
+  } else if (d.fast) {
+#pragma unroll
+    for (int m = 0; m < NCH; ++m)
+      if (t + T * m < nchunks)
+        *reinterpret_cast<uint2*>(qrow + (int64_t)(t + T * m) * 8) = pack8_codes<true, true>(v + m * 8, d);
+  } else {  // rare: a scale outside the fast range
+#pragma unroll
+    for (int m = 0; m < NCH; ++m)
+      if (t + T * m < nchunks)
+        *reinterpret_cast<uint2*>(qrow + (int64_t)(t + T * m) * 8) = pack8_codes<false, true>(v + m * 8, d);
+  }
 }
 
 // Packs four codes (low byte first) into one 32-bit word.

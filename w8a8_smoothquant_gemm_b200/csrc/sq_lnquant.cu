@@ -23,7 +23,8 @@ template <bool BF16, int MAXC, bool LN, bool PREFETCH, bool KEEP_Y>
 __global__ void __launch_bounds__(ROW_THREADS)
 ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
                        const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
-                       const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx) {
+                       const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
+                       const float* __restrict__ scale_in, int write_codes) {
   __shared__ float red[3 * (ROW_WARPS + 1)];
   const int nchunks = K / 8;
   RowChunks<BF16, MAXC> cur;
@@ -53,12 +54,12 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
       }
     }
     amax = block_max(amax, red + 2 * (ROW_WARPS + 1));
-    const float scale = __fdiv_rn(amax, 127.0f);
+    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, 127.0f);
     const SharedDivisor d(scale);
     if (threadIdx.x == 0) sx[m] = scale;
     int8_t* qrow = xq + m * (int64_t)K;
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
+    for (int i = 0; i < (write_codes ? MAXC : 0); ++i) {
       const int c = threadIdx.x + i * ROW_THREADS;
       if (c < nchunks) {
         float y[8];
@@ -71,12 +72,7 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
           if (LN) ln_chunk(f, mu, rstd, gamma_f, beta_f, c, y);
           else div_chunk(f, s, c, y);
         }
-        uint2 packed = make_uint2(0u, 0u);
-        if (scale != 0.0f) {
-          packed.x = pack4_low_bytes(code_bits(y[0], d), code_bits(y[1], d), code_bits(y[2], d), code_bits(y[3], d));
-          packed.y = pack4_low_bytes(code_bits(y[4], d), code_bits(y[5], d), code_bits(y[6], d), code_bits(y[7], d));
-        }
-        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = packed;
+        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false, true>(y, d);
       }
     }
     if (PREFETCH) cur = nxt;
@@ -91,7 +87,8 @@ template <bool BF16, int T, int NCH, bool LN>
 __global__ void __launch_bounds__(256, 2)
 ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
                       const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
-                      const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx) {
+                      const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
+                      const float* __restrict__ scale_in, int write_codes) {
   constexpr int G = 256 / T;
   __shared__ float red[G][24];  // per group: mean partials, variance partials, max
   extern __shared__ float rs[];  // plain mode: RN(1 / s_j), or 0 where s_j is outside the fast range
@@ -148,23 +145,26 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
     }
     float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
     amax = group_max<T>(amax, red[gid] + 16, t, gid);
-    const float scale = __fdiv_rn(amax, 127.0f);
+    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, 127.0f);
     if (t == 0) sx[m] = scale;
-    const SharedDivisor d(scale);
-    int8_t* qrow = xq + m * (int64_t)K;
-    if (d.fast) {
+    if (write_codes) store_row_codes<T, NCH>(v, t, nchunks, scale, scale_in != nullptr, xq + m * (int64_t)K);
+  }
+}
+
+// out[0] = max of v[0 .. n) (non-negative floats), one block.
+__global__ void __launch_bounds__(1024) max_of_vector_kernel(const float* __restrict__ v, int64_t n, float* out) {
+  __shared__ float red[32];
+  float m = 0.0f;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, v[i]);
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        const int c = t + T * i;
-        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<true>(v + i * 8, d);
-      }
-    } else {  // rare: a scale outside the fast range
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = red[threadIdx.x];
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        const int c = t + T * i;
-        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false>(v + i * 8, d);
-      }
-    }
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) out[0] = m;
   }
 }
 
@@ -175,7 +175,7 @@ namespace sqh {
 template <bool BF16, int T, int NCH, bool LN>
 static cudaError_t launch_group_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                   const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
-                                  cudaStream_t st) {
+                                  const float* scale_in, int write_codes, cudaStream_t st) {
   auto kern = sqk::ln_quant_group_kernel<BF16, T, NCH, LN>;
   const size_t smem = LN ? 0 : sizeof(float) * (size_t)K;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -186,18 +186,21 @@ static cudaError_t launch_group_t(const void* x, int64_t M, int K, int64_t ld_by
   constexpr int G = 256 / T;
   const int64_t blocks = (M + G - 1) / G;
   const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
-  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx);
+  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in,
+                                          write_codes);
   return cudaGetLastError();
 }
 
 template <bool BF16, int T>
 static cudaError_t launch_group_nch(int nch, const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                     const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
-                                    cudaStream_t st) {
-#define SQ_GRP(NCH)                                                                                          \
-  if (nch <= NCH)                                                                                            \
-    return gamma_f ? launch_group_t<BF16, T, NCH, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st) \
-                   : launch_group_t<BF16, T, NCH, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st);
+                                    const float* scale_in, int write_codes, cudaStream_t st) {
+#define SQ_GRP(NCH)                                                                                                \
+  if (nch <= NCH)                                                                                                  \
+    return gamma_f ? launch_group_t<BF16, T, NCH, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in, \
+                                                        write_codes, st)                                           \
+                   : launch_group_t<BF16, T, NCH, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in, \
+                                                         write_codes, st);
   SQ_GRP(1) SQ_GRP(2) SQ_GRP(4) SQ_GRP(8)
 #undef SQ_GRP
   return cudaErrorInvalidValue;
@@ -220,7 +223,7 @@ int pick_row_threads(int64_t K, int max_nch, int* nch) {
 template <bool BF16, int MAXC, bool LN>
 static cudaError_t launch_lnq_mode(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                    const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
-                                   cudaStream_t st) {
+                                   const float* scale_in, int write_codes, cudaStream_t st) {
   constexpr bool PF = BF16 && MAXC <= 4;      // register double buffer while it stays small
   constexpr bool KEEP = MAXC <= 8;            // y in registers (64 floats at most)
   auto kern = sqk::ln_smooth_quant_kernel<BF16, MAXC, LN, PF, KEEP>;
@@ -229,50 +232,79 @@ static cudaError_t launch_lnq_mode(const void* x, int64_t M, int K, int64_t ld_b
   if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(M, (int64_t)num_sms() * std::max(per_sm, 1));
   kern<<<(unsigned)grid, sqk::ROW_THREADS, 0, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq,
-                                                    sx);
+                                                    sx, scale_in, write_codes);
   return cudaGetLastError();
 }
 
 template <bool BF16, int MAXC>
 static cudaError_t launch_lnq_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                 const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
-                                cudaStream_t st) {
-  if (gamma_f) return launch_lnq_mode<BF16, MAXC, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st);
-  return launch_lnq_mode<BF16, MAXC, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, st);
+                                const float* scale_in, int write_codes, cudaStream_t st) {
+  if (gamma_f)
+    return launch_lnq_mode<BF16, MAXC, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st);
+  return launch_lnq_mode<BF16, MAXC, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st);
 }
 
 bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch);
 cudaError_t launch_rowpipe_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx, int T, int nch,
-                                 cudaStream_t st);
+                                 const float* scale_in, int write_codes, cudaStream_t st);
 
-cudaError_t launch_ln_smooth_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
-                                   const float* gamma_f, const float* beta_f, const float* s, float eps,
-                                   int8_t* xq, float* sx, cudaStream_t st) {
+// One pass of the row quantiser: per-token scales (scale_in == NULL) or a given per-tensor
+// scale; write_codes = 0 computes the per-token scales only.
+static cudaError_t launch_rows(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
+                               const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
+                               const float* scale_in, int write_codes, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   int pT = 0, pn = 0;
-  if (K <= 8192 && rowpipe_shape(K, bf16, 4, &pT, &pn))  // staged rows, 4 chunks per thread  // staged rows win up to 8192; beyond, register prefetch
-    return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, st);
+  if (K <= 8192 && rowpipe_shape(K, bf16, 4, &pT, &pn))  // staged rows, 4 chunks per thread
+    return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, scale_in, write_codes,
+                                st);
   int nch = 0;
   const int T = pick_row_threads(K, 8, &nch);
   if (T) {
     const int k = (int)K;
-#define SQ_T(TT)                                                                                      \
-  if (T == TT)                                                                                        \
-    return bf16 ? launch_group_nch<true, TT>(nch, x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, st)  \
-                : launch_group_nch<false, TT>(nch, x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, st);
+#define SQ_T(TT)                                                                                                    \
+  if (T == TT)                                                                                                      \
+    return bf16 ? launch_group_nch<true, TT>(nch, x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, \
+                                            st)                                                                     \
+                : launch_group_nch<false, TT>(nch, x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, scale_in,          \
+                                             write_codes, st);
     SQ_T(32) SQ_T(64) SQ_T(128) SQ_T(256)
 #undef SQ_T
   }
   const int need = (int)((K / 8 + sqk::ROW_THREADS - 1) / sqk::ROW_THREADS);
   const int k = (int)K;
-#define SQ_LNQ_CASE(C)                                                                                  \
-  if (need <= C)                                                                                        \
-    return bf16 ? launch_lnq_t<true, C>(x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, st)              \
-                : launch_lnq_t<false, (C > 16 ? 16 : C)>(x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, st);
+#define SQ_LNQ_CASE(C)                                                                                          \
+  if (need <= C)                                                                                                \
+    return bf16 ? launch_lnq_t<true, C>(x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st) \
+                : launch_lnq_t<false, (C > 16 ? 16 : C)>(x, M, k, ldb, gamma_f, beta_f, s, eps, xq, sx, scale_in,  \
+                                                         write_codes, st);
   SQ_LNQ_CASE(1) SQ_LNQ_CASE(2) SQ_LNQ_CASE(4) SQ_LNQ_CASE(8) SQ_LNQ_CASE(16) SQ_LNQ_CASE(24) SQ_LNQ_CASE(32)
 #undef SQ_LNQ_CASE
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_ln_smooth_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
+                                   const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                   int8_t* xq, float* sx, cudaStream_t st) {
+  return launch_rows(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, nullptr, 1, st);
+}
+
+cudaError_t launch_ln_smooth_quant_per_tensor(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
+                                              const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                              int static_scale, float* scale, int8_t* xq, float* sx,
+                                              cudaStream_t st) {
+  if (!static_scale) {
+    // per-token scales into sx, then scale = max_m sx[m] (= max |y| / 127: division by 127
+    // is monotone, so the max of the rounded quotients is the rounded quotient of the max)
+    cudaError_t e = launch_rows(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, nullptr, 0, st);
+    if (e != cudaSuccess) return e;
+    sqk::max_of_vector_kernel<<<1, 1024, 0, st>>>(sx, M, scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return launch_rows(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, scale, 1, st);
 }
 
 }  // namespace sqh

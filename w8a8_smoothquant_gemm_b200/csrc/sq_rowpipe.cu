@@ -25,7 +25,7 @@ template <bool BF16, int T, int NCH, int S, int MODE, bool POLL1 = false>
 __global__ void __launch_bounds__(256)
 rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, const float* __restrict__ vec_a,
                const float* __restrict__ vec_b, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
-               float* __restrict__ out, unsigned int* err) {
+               float* __restrict__ out, const float* __restrict__ scale_in, int write_codes, unsigned int* err) {
   constexpr int G = 256 / T;
   constexpr int ELT = BF16 ? 2 : 4;
   constexpr bool LN = MODE != ROW_PLAIN_QUANT;
@@ -181,23 +181,10 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
     float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])), fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
     amax = group_max<T>(amax, red[gid] + 16, t, gid);
     if (!LN && t == 0 && r + S * rstep < M) issue(slot, r + S * rstep);  // slot drained
-    const float scale = __fdiv_rn(amax, 127.0f);
+    // per-token scale, or the per-tensor scale handed in (then codes clamp at +-127)
+    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, 127.0f);
     if (t == 0) sx[r] = scale;
-    const SharedDivisor dv(scale);
-    int8_t* qrow = xq + r * (int64_t)K;
-    if (dv.fast) {
-#pragma unroll
-      for (int m = 0; m < NCH; ++m) {
-        const int c = t + T * m;
-        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<true>(v + m * 8, dv);
-      }
-    } else {  // rare: a scale outside the fast range
-#pragma unroll
-      for (int m = 0; m < NCH; ++m) {
-        const int c = t + T * m;
-        if (c < nchunks) *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false>(v + m * 8, dv);
-      }
-    }
+    if (write_codes) store_row_codes<T, NCH>(v, t, nchunks, scale, scale_in != nullptr, xq + r * (int64_t)K);
   }
 
   if (MODE == ROW_LN_CALIB) {
@@ -236,7 +223,8 @@ static size_t rowpipe_smem(int K, int elt, int G, int S) {
 
 template <bool BF16, int T, int NCH, int MODE, int S, bool POLL1>
 static cudaError_t launch_rowpipe_v(const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
-                                    const float* vb, float eps, int8_t* xq, float* sx, float* out, cudaStream_t st) {
+                                    const float* vb, float eps, int8_t* xq, float* sx, float* out, const float* scale_in,
+                                    int write_codes, cudaStream_t st) {
   constexpr int G = 256 / T;
   auto kern = sqk::rowpipe_kernel<BF16, T, NCH, S, MODE, POLL1>;
   const size_t smem = rowpipe_smem(K, BF16 ? 2 : 4, G, S);
@@ -247,7 +235,8 @@ static cudaError_t launch_rowpipe_v(const void* x, int64_t M, int K, int64_t ld_
   if (e != cudaSuccess) return e;
   const int64_t blocks = (M + G - 1) / G;
   const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
-  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, va, vb, eps, xq, sx, out, error_word_ptr());
+  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in,
+                                          write_codes, error_word_ptr());
   return cudaGetLastError();
 }
 
@@ -255,31 +244,37 @@ static cudaError_t launch_rowpipe_v(const void* x, int64_t M, int K, int64_t ld_
 // group waits in the hardware group barrier (measured best of {2, 3} slots x {one, all} pollers).
 template <bool BF16, int T, int NCH, int MODE>
 static cudaError_t launch_rowpipe_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
-                                    const float* vb, float eps, int8_t* xq, float* sx, float* out, cudaStream_t st) {
-  return launch_rowpipe_v<BF16, T, NCH, MODE, 2, true>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+                                    const float* vb, float eps, int8_t* xq, float* sx, float* out,
+                                    const float* scale_in, int write_codes, cudaStream_t st) {
+  return launch_rowpipe_v<BF16, T, NCH, MODE, 2, true>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in,
+                                                       write_codes, st);
 }
 
 template <bool BF16, int T, int MODE>
 static cudaError_t launch_rowpipe_nch(int nch, const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
                                       const float* vb, float eps, int8_t* xq, float* sx, float* out,
-                                      cudaStream_t st) {
-  if (nch <= 1) return launch_rowpipe_t<BF16, T, 1, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
-  if (nch <= 2) return launch_rowpipe_t<BF16, T, 2, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
-  if (nch <= 4) return launch_rowpipe_t<BF16, T, 4, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+                                      const float* scale_in, int write_codes, cudaStream_t st) {
+#define SQ_RP(N) launch_rowpipe_t<BF16, T, N, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in, write_codes, st)
+  if (nch <= 1) return SQ_RP(1);
+  if (nch <= 2) return SQ_RP(2);
+  if (nch <= 4) return SQ_RP(4);
   // calibration keeps at most 4 chunks per thread (its running maxima live in registers too)
   if (MODE == sqk::ROW_LN_CALIB) return cudaErrorInvalidValue;
   constexpr int N8 = MODE == sqk::ROW_LN_CALIB ? 4 : 8;
-  return launch_rowpipe_t<BF16, T, N8, MODE>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+  return SQ_RP(N8);
+#undef SQ_RP
 }
 
 template <int MODE>
 static cudaError_t launch_rowpipe_mode(bool bf16, int T, int nch, const void* x, int64_t M, int K, int64_t ld_bytes,
                                        const float* va, const float* vb, float eps, int8_t* xq, float* sx, float* out,
-                                       cudaStream_t st) {
-#define SQ_T(TT)                                                                                          \
-  if (T == TT)                                                                                            \
-    return bf16 ? launch_rowpipe_nch<true, TT, MODE>(nch, x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st) \
-                : launch_rowpipe_nch<false, TT, MODE>(nch, x, M, K, ld_bytes, va, vb, eps, xq, sx, out, st);
+                                       const float* scale_in, int write_codes, cudaStream_t st) {
+#define SQ_T(TT)                                                                                                 \
+  if (T == TT)                                                                                                   \
+    return bf16 ? launch_rowpipe_nch<true, TT, MODE>(nch, x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in,  \
+                                                    write_codes, st)                                             \
+                : launch_rowpipe_nch<false, TT, MODE>(nch, x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in, \
+                                                     write_codes, st);
   SQ_T(32) SQ_T(64) SQ_T(128) SQ_T(256)
 #undef SQ_T
   return cudaErrorInvalidValue;
@@ -295,20 +290,20 @@ bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch) {
 
 cudaError_t launch_rowpipe_quant(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx, int T, int nch,
-                                 cudaStream_t st) {
+                                 const float* scale_in, int write_codes, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   if (gamma_f)
     return launch_rowpipe_mode<sqk::ROW_LN_QUANT>(bf16, T, nch, x, M, (int)K, ldb, gamma_f, beta_f, eps, xq, sx,
-                                                  nullptr, st);
+                                                  nullptr, scale_in, write_codes, st);
   return launch_rowpipe_mode<sqk::ROW_PLAIN_QUANT>(bf16, T, nch, x, M, (int)K, ldb, s, nullptr, eps, xq, sx, nullptr,
-                                                   st);
+                                                   scale_in, write_codes, st);
 }
 
 cudaError_t launch_rowpipe_calib(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx, const float* gamma,
                                  const float* beta, float eps, float* out, int T, int nch, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   return launch_rowpipe_mode<sqk::ROW_LN_CALIB>(bf16, T, nch, x, rows, (int)K, ldb, gamma, beta, eps, nullptr, nullptr,
-                                                out, st);
+                                                out, nullptr, 1, st);
 }
 
 }  // namespace sqh
