@@ -196,6 +196,86 @@ def test_calib_ln_absmax(rows, K):
     assert np.array_equal(host(got), O.calib_ln_absmax(c.x, c.gamma, c.beta))
 
 
+# ----------------------------------------------------------------------------- prefill-sized row counts
+# From about a thousand rows on, rows of the model widths go to one-warp-per-row kernels
+# (chunk pairs on packed binary32); these cases cover every width they take, with a ragged
+# row count, a padded leading dimension and the degenerate rows.
+PAIR_WIDTHS = [512, 1024, 2048, 4096, 8192, 12288, 14336]
+
+
+def _many_rows(M, K, seed):
+    c = sq_inputs.make_case(M, K, 8, seed, beta_std=0.05)
+    c.x[1] = 0  # all-zero row
+    # a row of tiny values: in plain mode its scale falls below 2^-90, where the shared-divisor
+    # quotient takes the correctly rounded division instead
+    c.x[2] = sq_inputs.to_bf16_bits(O.bf16_to_f32(c.x[2]) * np.float32(2.0 ** -100))
+    return c
+
+
+@pytest.mark.parametrize("K", PAIR_WIDTHS)
+@pytest.mark.parametrize("mode", ["ln", "plain"])
+def test_ln_smooth_quant_many_rows(K, mode):
+    M = 1031
+    c = _many_rows(M, K, 11 * K + 3)
+    s = np.exp(np.random.default_rng(K + 5).uniform(-1, 3, K)).astype(np.float32)
+    xd = dev(padded(c.x, 16))[:, :K]
+    if mode == "ln":
+        gf, bf = (c.gamma / s).astype(np.float32), (c.beta / s).astype(np.float32)
+        xq, sx = sq.sq_ln_smooth_quant(xd, gamma_f=dev(gf), beta_f=dev(bf))
+        r_xq, r_sx = O.ln_smooth_quant(c.x, gamma_f=gf, beta_f=bf)
+    else:
+        xq, sx = sq.sq_ln_smooth_quant(xd, s=dev(s))
+        r_xq, r_sx = O.ln_smooth_quant(c.x, s=s)
+        assert r_sx[2] < 2.0 ** -90 and r_sx[1] == 0
+    assert np.array_equal(host(sx), r_sx)
+    assert np.array_equal(host(xq), r_xq)
+
+
+@pytest.mark.parametrize("K", [4096, 14336])
+def test_plain_quant_many_rows_divisor_outside_fast_range(K):
+    """A smoothing factor below 2^-90: every division of that launch is correctly rounded."""
+    M = 1030
+    c = _many_rows(M, K, K + 17)
+    s = np.exp(np.random.default_rng(K + 6).uniform(-1, 3, K)).astype(np.float32)
+    s[5] = np.float32(2.0 ** -100)
+    xq, sx = sq.sq_ln_smooth_quant(dev(c.x), s=dev(s))
+    r_xq, r_sx = O.ln_smooth_quant(c.x, s=s)
+    assert np.array_equal(host(sx), r_sx)
+    assert np.array_equal(host(xq), r_xq)
+
+
+@pytest.mark.parametrize("K", PAIR_WIDTHS)
+@pytest.mark.parametrize("mode", ["ln", "plain"])
+def test_per_tensor_many_rows(K, mode):
+    """Per-tensor scales (dynamic, then static at half of it: clamping) through the same kernels."""
+    M = 1029
+    c = sq_inputs.make_case(M, K, 8, 13 * K + 1, beta_std=0.05)
+    s = np.exp(np.random.default_rng(K + 7).uniform(-1, 3, K)).astype(np.float32)
+    kw = dict(gamma_f=(c.gamma / s).astype(np.float32)) if mode == "ln" else dict(s=s)
+    dkw = {k: dev(v) for k, v in kw.items()}
+    xq, sx, sc = sq.sq_ln_smooth_quant_per_tensor(dev(c.x), **dkw)
+    r_xq, r_sx, r_sc = O.ln_smooth_quant_per_tensor(c.x, **kw)
+    assert host(sc)[0] == np.float32(r_sc)
+    assert np.array_equal(host(sx), r_sx) and np.array_equal(host(xq), r_xq)
+    static = np.float32(r_sc * 0.5)
+    xq, sx, _ = sq.sq_ln_smooth_quant_per_tensor(dev(c.x), scale=dev(np.array([static], np.float32)), static=True,
+                                                 **dkw)
+    r_xq, r_sx, _ = O.ln_smooth_quant_per_tensor(c.x, static_scale=float(static), **kw)
+    assert np.array_equal(host(sx), r_sx) and np.array_equal(host(xq), r_xq)
+    assert (np.abs(r_xq) == 127).sum() > 0
+
+
+@pytest.mark.parametrize("rows,K", [(1030, 512), (1100, 1024), (1027, 2048), (2051, 4096), (1500, 8192)])
+def test_calib_ln_absmax_many_rows(rows, K):
+    c = _many_rows(rows, K, rows + 3 * K)
+    x = dev(padded(c.x, 8))[:, :K]
+    got = sq.sq_calib_ln_absmax(x, dev(c.gamma), dev(c.beta))
+    ref = O.calib_ln_absmax(c.x, c.gamma, c.beta)
+    assert np.array_equal(host(got), ref)
+    sq.sq_calib_ln_absmax(x, dev(c.gamma), dev(c.beta), out=got, accumulate=True)
+    assert np.array_equal(host(got), ref)
+
+
 # ----------------------------------------------------------------------------- GEMM
 def random_codes(rng, rows, K, extreme_row=None):
     q = rng.integers(-127, 128, (rows, K), dtype=np.int64).astype(np.int8)

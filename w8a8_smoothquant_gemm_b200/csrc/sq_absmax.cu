@@ -337,6 +337,9 @@ static cudaError_t launch_calib_ln_t(const void* x, int64_t rows, int K, int64_t
 }
 
 int pick_row_threads(int64_t K, int max_nch, int* nch);
+bool rowpair_supported(int64_t K, bool bf16, bool calib, int64_t rows);
+cudaError_t launch_rowpair_calib(const void* x, int64_t rows, int64_t K, int64_t ldx, const float* gamma,
+                                 const float* beta, float eps, float* out, cudaStream_t st);
 bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch);
 cudaError_t launch_rowpipe_calib(const void* x, bool bf16, int64_t rows, int64_t K, int64_t ldx, const float* gamma,
                                  const float* beta, float eps, float* out, int T, int nch, cudaStream_t st);
@@ -372,6 +375,8 @@ cudaError_t launch_calib_ln_absmax(const void* x, bool bf16, int64_t rows, int64
     if (e != cudaSuccess) return e;
   }
   const int64_t ldb = ld * (bf16 ? 2 : 4);
+  if (rowpair_supported(K, bf16, true, rows))  // chunk-pair rows of the model widths
+    return launch_rowpair_calib(x, rows, K, ld, gamma, beta, eps, out, st);
   int pT = 0, pn = 0;
   if (rowpipe_shape(K, bf16, 4, &pT, &pn))
     return launch_rowpipe_calib(x, bf16, rows, K, ld, gamma, beta, eps, out, pT, pn, st);

@@ -250,12 +250,19 @@ cudaError_t launch_rowpipe_quant(const void* x, bool bf16, int64_t M, int64_t K,
                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx, int T, int nch,
                                  const float* scale_in, int write_codes, cudaStream_t st);
 
+bool rowpair_supported(int64_t K, bool bf16, bool calib, int64_t rows);
+cudaError_t launch_rowpair_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
+                                 const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
+                                 const float* scale_in, int write_codes, cudaStream_t st);
+
 // One pass of the row quantiser: per-token scales (scale_in == NULL) or a given per-tensor
 // scale; write_codes = 0 computes the per-token scales only.
 static cudaError_t launch_rows(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                                const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                const float* scale_in, int write_codes, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
+  if (rowpair_supported(K, bf16, false, M))  // chunk-pair rows of the model widths
+    return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st);
   int pT = 0, pn = 0;
   if (K <= 8192 && rowpipe_shape(K, bf16, 4, &pT, &pn))  // staged rows, 4 chunks per thread
     return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, scale_in, write_codes,
