@@ -56,6 +56,16 @@ def lib() -> ctypes.CDLL:
         L.sqo_quant_per_tensor.restype = None
         L.sqo_w8a8_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I, I64]
         L.sqo_w8a8_gemm.restype = I64
+        L.sqo_e4m3_encode.argtypes = [F]
+        L.sqo_e4m3_encode.restype = ctypes.c_uint8
+        L.sqo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.sqo_e4m3_decode.restype = F
+        L.sqo_fold_quant_weights_fp8.argtypes = [P, I, I64, I64, I64, P, P, P, P, P, P, P]
+        L.sqo_fold_quant_weights_fp8.restype = None
+        L.sqo_ln_smooth_quant_fp8.argtypes = [P, I, I64, I64, I64, P, P, P, F, P, P]
+        L.sqo_ln_smooth_quant_fp8.restype = None
+        L.sqo_fp8_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, P, I, I64]
+        L.sqo_fp8_gemm.restype = None
         L.sqo_f32_to_bf16.argtypes = [F]
         L.sqo_f32_to_bf16.restype = ctypes.c_uint16
         L.sqo_num_threads.argtypes = []
@@ -215,6 +225,65 @@ def w8a8_gemm(xq: np.ndarray, sx: np.ndarray, wq: np.ndarray, sw: np.ndarray, ou
     if over:
         raise OverflowError(f"{over} accumulators outside int32")
     return y
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3) variant
+def e4m3_encode(v) -> np.ndarray:
+    """float32 values -> E4M3 codes (uint8): nearest even, saturating at +-448."""
+    v = np.asarray(v, dtype=np.float32)
+    f = lib().sqo_e4m3_encode
+    return np.array([f(float(a)) for a in v.reshape(-1)], np.uint8).reshape(v.shape)
+
+
+def e4m3_decode(c) -> np.ndarray:
+    """E4M3 codes (uint8) -> float32 values (exact)."""
+    c = np.asarray(c, dtype=np.uint8)
+    f = lib().sqo_e4m3_decode
+    return np.array([f(int(a)) for a in c.reshape(-1)], np.float32).reshape(c.shape)
+
+
+def fold_quant_weights_fp8(W: np.ndarray, s: np.ndarray, gamma=None, beta=None):
+    """W [K, N] -> (Wq [N, K] E4M3 codes, sw [N] = column max / 448, gamma', beta')."""
+    W, s = _c(W), _c(s, np.float32)
+    K, N = W.shape
+    wq = np.empty((N, K), np.uint8)
+    sw = np.empty(N, np.float32)
+    gamma, beta = _c(gamma, np.float32), _c(beta, np.float32)
+    gf = np.empty(K, np.float32) if gamma is not None else None
+    bf = np.empty(K, np.float32) if beta is not None else None
+    lib().sqo_fold_quant_weights_fp8(_ptr(W), _dtype_code(W), K, N, N, _ptr(s), _ptr(gamma), _ptr(beta),
+                                     _ptr(wq), _ptr(sw), _ptr(gf), _ptr(bf))
+    return wq, sw, gf, bf
+
+
+def ln_smooth_quant_fp8(x: np.ndarray, gamma_f=None, beta_f=None, s=None, eps: float = 1e-5):
+    """Per-token E4M3 of LN(x) (folded gamma', beta') or of x / s; sx = row max / 448."""
+    if (gamma_f is None) == (s is None):
+        raise ValueError("exactly one of gamma_f (LayerNorm mode) and s (plain mode) is given")
+    x = _c(x)
+    M, K = x.shape
+    xq = np.empty((M, K), np.uint8)
+    sx = np.empty(M, np.float32)
+    lib().sqo_ln_smooth_quant_fp8(_ptr(x), _dtype_code(x), M, K, K, _ptr(_c(gamma_f, np.float32)),
+                                  _ptr(_c(beta_f, np.float32)), _ptr(_c(s, np.float32)), float(eps),
+                                  _ptr(xq), _ptr(sx))
+    return xq, sx
+
+
+def fp8_gemm(xq: np.ndarray, sx: np.ndarray, wq: np.ndarray, sw: np.ndarray, out: str = "bf16"):
+    """Exact accumulators acc = dec(xq) @ dec(wq)^T (float64) and the output
+    ((float)acc * sx) * sw as 'f32' or 'bf16' bits.  Returns (acc, y)."""
+    xq, wq = _c(xq, np.uint8), _c(wq, np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError("xq and wq disagree on K")
+    code, dt = {"f32": (F32, np.float32), "bf16": (BF16, np.uint16)}[out]
+    acc = np.empty((M, N), np.float64)
+    y = np.empty((M, N), dt)
+    lib().sqo_fp8_gemm(_ptr(xq), _ptr(_c(sx, np.float32)), _ptr(wq), _ptr(_c(sw, np.float32)), M, N, K,
+                       _ptr(acc), _ptr(y), code, N)
+    return acc, y
 
 
 # ----------------------------------------------------------------------------- binary64 definitions

@@ -22,6 +22,14 @@
  *   [INT8GEMM] "4.2 W8A8 量化与 SmoothQuant", intro (GEMM entirely on INT8 tensor cores);
  *             "量化：只压权重…", SmoothQuant section (per-token / per-channel scales
  *             factor out of the sum; per-input-channel activation scales do not).
+ *   [FP8]     "量化：只压权重，与训练后量化（PTQ）", the W8A8-FP8 rows of the decode
+ *             roofline (FP8 tensor-core peak twice BF16) and "4.2 W8A8 量化与
+ *             SmoothQuant", closing questions (FP8 as the 8-bit format that may need no
+ *             explicit smoothing).  The pages do not define the FP8 encoding; the reading
+ *             taken is E4M3 of the OCP 8-bit floating point specification (OFP8): bias 7,
+ *             3 mantissa bits, no infinities, S.1111.111 = NaN, largest finite 448, with the
+ *             same symmetric scheme as INT8 -- scale = max|.| / 448 and code = E4M3 of
+ *             RN(v / scale), round to nearest even, saturating at +-448.
  *
  * Readings where the pages are silent (each is a convention shared with the GPU
  * path so that results can be compared bit for bit; no page value checks them,
@@ -363,6 +371,128 @@ void sqo_quant_per_tensor(const float* y, int64_t n, int8_t* q, float* scale_out
   const float scale = amax / 127.0f;
   for (int64_t i = 0; i < n; ++i) q[i] = quant_code(y[i], scale);
   *scale_out = scale;
+}
+
+/* ---------------------------------------------------------------------------
+ * FP8 E4M3 codes  [FP8]
+ *   decode: e = bits 6..3, m = bits 2..0; e = 0: (m / 8) 2^-6; else (1 + m / 8) 2^(e-7);
+ *           e = 15 and m = 7: NaN
+ *   encode: round to nearest even on the E4M3 grid; magnitudes that round above 448
+ *           saturate to 448; NaN -> 0x7F; -0 keeps its sign
+ * ------------------------------------------------------------------------- */
+float sqo_e4m3_decode(uint8_t c) {
+  const int e = (c >> 3) & 15, m = c & 7;
+  float v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexpf((float)m, -9);
+  else v = ldexpf((float)(8 + m), e - 10);
+  return (c & 0x80) ? -v : v;
+}
+
+uint8_t sqo_e4m3_encode(float v) {
+  if (isnan(v)) return 0x7F;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const float a = fabsf(v);
+  if (a >= 448.0f) return sign | 0x7E;
+  if (a < 0x1p-6f) {                       /* subnormal grid, spacing 2^-9 */
+    const float q = rintf(ldexpf(a, 9));   /* 0 .. 8; 8 is the smallest normal, code 8 */
+    return sign | (uint8_t)q;
+  }
+  int e;
+  frexpf(a, &e);                           /* a = f 2^e, f in [0.5, 1) */
+  e -= 1;                                  /* a in [2^e, 2^(e+1)), e in -6 .. 8 */
+  float q = rintf(ldexpf(a, 3 - e));       /* 8 .. 16 steps of 2^(e-3) */
+  if (q == 16.0f) {
+    q = 8.0f;
+    e += 1;
+  }
+  if (e > 8 || (e == 8 && q > 14.0f)) return sign | 0x7E; /* above 448: saturate */
+  return sign | (uint8_t)(((e + 7) << 3) | ((int)q - 8));
+}
+
+/* E4M3 code of v with a shared scale: RN(v / scale) on the E4M3 grid; scale 0 -> +0. */
+static uint8_t fp8_code(float v, float scale) {
+  if (scale == 0.0f) return 0;
+  return sqo_e4m3_encode(v / scale);
+}
+
+/* Fold + per-output-channel FP8 weights: as sqo_fold_quant_weights with
+ * sw[k] = max_j |W'[j, k]| / 448 and E4M3 codes.  [SQ-eq], [SQ-LN], [SQ-pipe], [FP8] */
+void sqo_fold_quant_weights_fp8(const void* W, int dt, int64_t K, int64_t N, int64_t ldw,
+                                const float* s, const float* gamma, const float* beta,
+                                uint8_t* Wq, float* sw, float* gamma_f, float* beta_f) {
+#pragma omp parallel for schedule(static)
+  for (int64_t k = 0; k < N; ++k) {
+    float m = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+      float a = fabsf(s[j] * load_elt(W, dt, j * ldw + k));
+      if (a > m) m = a;
+    }
+    const float scale = m / 448.0f;
+    sw[k] = scale;
+    for (int64_t j = 0; j < K; ++j) Wq[k * K + j] = fp8_code(s[j] * load_elt(W, dt, j * ldw + k), scale);
+  }
+  if (gamma && gamma_f)
+    for (int64_t j = 0; j < K; ++j) gamma_f[j] = gamma[j] / s[j];
+  if (beta && beta_f)
+    for (int64_t j = 0; j < K; ++j) beta_f[j] = beta[j] / s[j];
+}
+
+/* Fused LayerNorm -> X diag(s)^-1 -> per-token FP8: as sqo_ln_smooth_quant with
+ * sx_m = max_j |y_mj| / 448 and E4M3 codes.  [SQ-LN], [SQ-pipe], [FP8] */
+void sqo_ln_smooth_quant_fp8(const void* x, int dt, int64_t M, int64_t K, int64_t ldx,
+                             const float* gamma_f, const float* beta_f, const float* s,
+                             float eps, uint8_t* xq, float* sx) {
+#pragma omp parallel
+  {
+    float* xr = (float*)malloc(sizeof(float) * (size_t)K);
+    float* yr = (float*)malloc(sizeof(float) * (size_t)K);
+    float* tmp = (float*)malloc(sizeof(float) * (size_t)K);
+#pragma omp for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+      for (int64_t j = 0; j < K; ++j) xr[j] = load_elt(x, dt, m * ldx + j);
+      if (gamma_f) {
+        layernorm_row(xr, K, gamma_f, beta_f, eps, yr, tmp);
+      } else {
+        for (int64_t j = 0; j < K; ++j) yr[j] = xr[j] / s[j];
+      }
+      float amax = 0.0f;
+      for (int64_t j = 0; j < K; ++j) {
+        const float a = fabsf(yr[j]);
+        if (a > amax) amax = a;
+      }
+      const float scale = amax / 448.0f;
+      sx[m] = scale;
+      for (int64_t j = 0; j < K; ++j) xq[m * K + j] = fp8_code(yr[j], scale);
+    }
+    free(xr); free(yr); free(tmp);
+  }
+}
+
+/* FP8 x FP8 GEMM with the dequant epilogue  [FP8], [INT8GEMM]
+ *   acc[m, n] = sum_j dec(xq[m, j]) dec(wq[n, j]), exact: every product of two E4M3 values
+ *   has at most 8 significant bits and lies in [2^-18, 448^2], so a binary64 running sum
+ *   of up to 2^16 of them never rounds.
+ *   acc_out (optional): the exact accumulators;  y: ((float)acc * sx[m]) * sw[n] in
+ *   binary32 (F32) or its bfloat16 (BF16), (float)acc being the rounded exact sum. */
+void sqo_fp8_gemm(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                  int64_t M, int64_t N, int64_t K, double* acc_out, void* y, int ydt, int64_t ldy) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j)
+        acc += (double)sqo_e4m3_decode(xq[m * K + j]) * (double)sqo_e4m3_decode(wq[n * K + j]);
+      if (acc_out) acc_out[m * N + n] = acc;
+      if (y) {
+        const float v = ((float)acc * sx[m]) * sw[n];
+        if (ydt == SQO_BF16)
+          ((uint16_t*)y)[m * ldy + n] = f32_to_bf16(v);
+        else
+          ((float*)y)[m * ldy + n] = v;
+      }
+    }
+  }
 }
 
 /* ---------------------------------------------------------------------------

@@ -394,3 +394,100 @@ def test_per_tensor_layernorm_mode_uses_the_same_layernorm():
     assert scale == np.float32(np.max(np.abs(y))) / np.float32(127.0)
     q2, _ = O.quant_per_tensor(y)
     assert np.array_equal(xq, q2)
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3) variant
+# The pages name FP8 W8A8 (the FP8 tensor-core peak is twice BF16's) without fixing the
+# encoding; the reading is E4M3 of the OCP 8-bit floating point specification, and these
+# pins hold the oracle's encoder and decoder to torch's float8_e4m3fn, an independent
+# implementation of the same format.
+def _torch_e4m3(v: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_decode_every_code_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    got = O.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin].view(np.uint32), ref[fin].view(np.uint32))
+    assert np.isnan(got).sum() == 2 and got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+def test_e4m3_encode_grid_midpoints_and_random_values_match_torch():
+    grid = O.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8)).astype(np.float64)  # 0 .. 448
+    mids = (grid[:-1] + grid[1:]) / 2                      # ties: nearest even code
+    quarter = grid[:-1] + (grid[1:] - grid[:-1]) / 4
+    rng = np.random.default_rng(3)
+    rand = np.concatenate([rng.uniform(0, 463.9, 4000), np.exp(rng.uniform(np.log(2.0 ** -12), np.log(463.0), 4000))])
+    v = np.concatenate([grid, mids, quarter, rand]).astype(np.float32)
+    v = np.concatenate([v, -v])
+    assert np.array_equal(O.e4m3_encode(v), _torch_e4m3(v))
+    assert np.array_equal(O.e4m3_encode(O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))), np.arange(0x7F))
+
+
+def test_e4m3_saturates_at_the_largest_finite_value():
+    v = np.array([448.0, 463.9, 464.0, 500.0, 1e30, -470.0], np.float32)
+    assert O.e4m3_encode(v).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+
+
+def test_fp8_fold_per_output_channel():
+    c = sq_inputs.make_case(4, 96, 40, 12)
+    s = np.exp(np.random.default_rng(4).uniform(-1, 1, 96)).astype(np.float32)
+    wq, sw, _, _ = O.fold_quant_weights_fp8(c.W, s)
+    Wp = (s[:, None] * O.bf16_to_f32(c.W)).astype(np.float32)          # W' = diag(s) W, [K, N]
+    assert np.array_equal(sw, np.max(np.abs(Wp), axis=0) / np.float32(448.0))
+    dec = O.e4m3_decode(wq).astype(np.float64)                           # [N, K]
+    assert np.all(np.max(np.abs(dec), axis=1) == 448.0)                  # every column reaches the top code
+    err = np.abs(dec * sw[:, None] - Wp.T.astype(np.float64))
+    # half an E4M3 step: 2^-4 relative for normal codes, 2^-10 of the scale below 2^-6
+    assert np.all(err <= np.maximum(np.abs(Wp.T) * 2.0 ** -4, 2.0 ** -10 * sw[:, None]) * (1 + 1e-6))
+
+
+def test_fp8_per_token_codes_follow_the_definition():
+    c = sq_inputs.make_case(9, 128, 8, 13)
+    s = np.exp(np.random.default_rng(5).uniform(-1, 2, 128)).astype(np.float32)
+    xq, sx = O.ln_smooth_quant_fp8(c.x, s=s)
+    y = (O.bf16_to_f32(c.x) / s[None, :]).astype(np.float32)
+    ref_sx = np.max(np.abs(y), axis=1) / np.float32(448.0)
+    assert np.array_equal(sx, ref_sx)
+    q = (y / ref_sx[:, None]).astype(np.float32)
+    assert np.array_equal(xq, _torch_e4m3(q))                            # |q| <= 448: torch's rounding applies
+    xl, sl = O.ln_smooth_quant_fp8(c.x, gamma_f=c.gamma)
+    yl = O.layernorm(c.x, c.gamma)
+    assert np.array_equal(sl, np.max(np.abs(yl), axis=1) / np.float32(448.0))
+    assert np.array_equal(xl, _torch_e4m3((yl / sl[:, None]).astype(np.float32)))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 16), (3, 5, 64), (7, 6, 200)])
+def test_fp8_gemm_accumulator_is_the_exact_sum(M, N, K):
+    import fractions
+    rng = np.random.default_rng(M * N + K)
+    fin = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    xq = rng.choice(fin, (M, K)).astype(np.uint8)
+    wq = rng.choice(fin, (N, K)).astype(np.uint8)
+    xq[0, :4] = 0x7E
+    wq[0, :4] = 0xFE                                                     # -448 * 448 products
+    acc, y = O.fp8_gemm(xq, np.ones(M, np.float32), wq, np.ones(N, np.float32), "f32")
+    dx, dw = O.e4m3_decode(xq), O.e4m3_decode(wq)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(fractions.Fraction(float(a)) * fractions.Fraction(float(b)) for a, b in zip(dx[m], dw[n]))
+            assert fractions.Fraction(acc[m, n]) == exact
+            assert y[m, n] == np.float32(float(exact))
+
+
+def test_fp8_smoothquant_linear_error_is_small():
+    """Smoothing + E4M3 codes on the outlier case: the dequantised linear stays within a few
+    E4M3 steps of XW (3 mantissa bits: per-element error below 2^-4 relative)."""
+    c = sq_inputs.tiny_case()
+    x = O.bf16_to_f32(c.x) if c.x.dtype == np.uint16 else c.x
+    W = O.bf16_to_f32(c.W) if c.W.dtype == np.uint16 else c.W
+    s = O.smooth_factors(O.calib_absmax(x, 0), O.calib_absmax(W, 1), 0.5)
+    wq, sw, _, _ = O.fold_quant_weights_fp8(W, s)
+    xq, sx = O.ln_smooth_quant_fp8(x, s=s)
+    acc, _ = O.fp8_gemm(xq, sx, wq, sw, "f32")
+    yq = acc * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
+    Y = x.astype(np.float64) @ W.astype(np.float64)
+    assert _rel_fro(yq, Y) < 2.0 ** -4
