@@ -521,8 +521,20 @@ def run_kernel(args):
             nxt[0] += 1
         return call
 
+    if args.kernel == "gemm8":
+        # the FP8 variant on the same linear: E4M3 codes of the same smoothed operands
+        wq8, sw8, gf8, _ = sq.sq_fold_quant_weights_fp8(L.W, L.s, L.gamma)
+        xq8, sx8 = sq.sq_ln_smooth_quant_fp8(L.x, gamma_f=gf8)
+        copies8 = [(xq8.clone(), wq8.clone(), torch.empty_like(L.y)) for _ in range(n_copies)]
+
+    def gemm8_call():
+        xq, wq, y = copies8[rot[0] % n_copies]
+        rot[0] += 1
+        sq.sq_w8a8_gemm_fp8(xq, sx8, wq, sw8, y=y, workspace=L.ws)
+
     calls = {
         "gemm": (gemm_call, gemm_bytes, 2.0 * M * N * K),
+        "gemm8": (gemm8_call, gemm_bytes, 2.0 * M * N * K),
         "fold": (rotated(lambda: sq.sq_fold_quant_weights(pick(ws), L.s, L.gamma, wq=pick(wq_out), sw=L.sw,
                                                           gamma_f=L.gf)), L.bytes_fold(), 0.0),
         "lnquant": (rotated(lambda: sq.sq_ln_smooth_quant(pick(xs), gamma_f=L.gf, xq=pick(xq_out), sx=L.sx)),
@@ -540,7 +552,7 @@ def run_kernel(args):
     # device time per call: `steps` calls captured in one CUDA graph (no host launch cost in
     # the timed region), replayed a few times; the median replay / steps
     reps = 5
-    if args.kernel == "gemm":
+    if args.kernel in ("gemm", "gemm8"):
         args.steps = max(args.steps, n_copies)
     else:
         args.steps = max(args.steps, len(xs), len(ws))
@@ -580,7 +592,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=("gemm", "fold", "lnquant", "quant", "calib", "wabsmax", "xabsmax"),
+    ap.add_argument("--kernel", choices=("gemm", "gemm8", "fold", "lnquant", "quant", "calib", "wabsmax", "xabsmax"),
                     help="run only this kernel on --shape M,N,K (profiling aid; prints no bench line)")
     ap.add_argument("--shape", default="2048,4096,4096")
     args = ap.parse_args()

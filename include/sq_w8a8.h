@@ -177,6 +177,46 @@ sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* sx, const int8_t* 
                                int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                                void* stream);
 
+/* ------------------------------------------------------------------------------------------
+ * FP8 variant.  "量化：只压权重，与训练后量化（PTQ）" (decode roofline: W8A8 in FP8 runs on tensor
+ * cores with twice the BF16 peak) and "4.2 W8A8 量化与 SmoothQuant" (closing questions: FP8 as
+ * the 8-bit format) name FP8 W8A8 without fixing the encoding.  The library reads it as E4M3
+ * of the OCP 8-bit floating point specification (OFP8): sign, 4 exponent bits (bias 7),
+ * 3 mantissa bits, no infinities, 0x7F / 0xFF = NaN, largest finite 448.  The scheme is the
+ * INT8 one with 448 in place of 127: scale = max|.| / 448 (binary32, correctly rounded) and
+ * code = E4M3(RN(v / scale)), round to nearest even, saturating at +-448; a zero scale gives
+ * +0 codes.  Codes are stored as uint8_t bit patterns.
+ * ------------------------------------------------------------------------------------------ */
+
+/* sq_fold_quant_weights_fp8 -- sq_fold_quant_weights with E4M3 weights:
+ *   sw[k] = max_j |W'[j, k]| / 448;  Wq[k, j] = E4M3(RN(W'[j, k] / sw[k])).
+ *   Every argument has the meaning, layout, ownership and checks of sq_fold_quant_weights
+ *   (Wq: uint8 [N, K], K contiguous, 16-byte aligned). */
+sq_status sq_fold_quant_weights_fp8(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                                    const float* s, const float* gamma, const float* beta,
+                                    uint8_t* Wq, float* sw, float* gamma_f, float* beta_f, void* stream);
+
+/* sq_ln_smooth_quant_fp8 -- sq_ln_smooth_quant with per-token E4M3 codes:
+ *   sx[m] = max_j |y[m, j]| / 448;  xq[m, j] = E4M3(RN(y[m, j] / sx[m])).
+ *   y, the two modes and every argument as for sq_ln_smooth_quant (xq: uint8 [M, K]). */
+sq_status sq_ln_smooth_quant_fp8(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                 const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                 uint8_t* xq, float* sx, void* stream);
+
+/* sq_w8a8_gemm_fp8 -- E4M3 x E4M3 GEMM on the tcgen05 tensor cores (kind::f8f6f4) with the
+ * same dequant epilogue:
+ *   acc[m, n] = sum_j dec(xq[m, j]) dec(wq[n, j])   accumulated in binary32 by the tensor
+ *              cores (every product is exact; the order and rounding of the sum are the
+ *              hardware's, so acc is within the binary32 summation error bound of the exact
+ *              sum, not bit-identical to it)
+ *   ydt = SQ_BF16: y[m, n] = bf16_rne((acc[m, n] * sx[m]) * sw[n]);  SQ_F32: the same in fp32.
+ *   SQ_I32 is invalid.  Operands, leading dimension, alignment, K limit and workspace as for
+ *   sq_w8a8_gemm; the workspace size is sq_w8a8_gemm_workspace_size(M, N, K) (fp32
+ *   partials, summed in split order). */
+sq_status sq_w8a8_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                           int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
+                           void* workspace, size_t ws_bytes, void* stream);
+
 /* Reads (and with clear != 0 resets) the device-side error word of the current device:
  * 0 when no kernel gave up on a bounded wait.  Synchronises `stream`. */
 sq_status sq_device_error(unsigned int* code, int clear, void* stream);

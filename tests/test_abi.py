@@ -42,7 +42,7 @@ def test_status_strings_and_version():
     L = sq.lib()
     assert L.sq_status_string(0) == b"SQ_OK"
     assert L.sq_status_string(5) == b"SQ_ERR_WORKSPACE"
-    assert L.sq_abi_version() == 100
+    assert L.sq_abi_version() == 101
 
 
 # fake, never dereferenced device addresses with chosen alignment

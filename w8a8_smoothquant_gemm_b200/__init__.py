@@ -9,6 +9,8 @@ if the library cannot be loaded, every call raises.
 Pipeline ("4.2 W8A8 量化与 SmoothQuant", sec. 7.1):
   offline:  sq_calib_absmax / sq_calib_ln_absmax -> sq_smooth_factors -> sq_fold_quant_weights
   runtime:  sq_ln_smooth_quant -> sq_w8a8_gemm
+FP8 (E4M3) variant of the quantised steps: sq_fold_quant_weights_fp8, sq_ln_smooth_quant_fp8,
+sq_w8a8_gemm_fp8.
 """
 from __future__ import annotations
 
@@ -54,6 +56,9 @@ def lib() -> ctypes.CDLL:
             "sq_ln_smooth_quant_per_tensor": [P, I, I64, I64, I64, P, P, P, F, I, P, P, P, P],
             "sq_w8a8_gemm": [P, P, P, P, I64, I64, I64, P, I, I64, P, SZ, P],
             "sq_device_error": [P, I, P],
+            "sq_fold_quant_weights_fp8": [P, I, I64, I64, I64, P, P, P, P, P, P, P, P],
+            "sq_ln_smooth_quant_fp8": [P, I, I64, I64, I64, P, P, P, F, P, P, P],
+            "sq_w8a8_gemm_fp8": [P, P, P, P, I64, I64, I64, P, I, I64, P, SZ, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -252,6 +257,78 @@ def sq_w8a8_gemm(xq: torch.Tensor, sx: torch.Tensor | None, wq: torch.Tensor, sw
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("sq_w8a8_gemm", lib().sq_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
                                               y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))
+    return y
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3) variant
+# Codes are uint8 tensors holding E4M3 bit patterns (view them as torch.float8_e4m3fn if
+# wanted); scales are max / 448.
+def sq_fold_quant_weights_fp8(W: torch.Tensor, s: torch.Tensor, gamma: torch.Tensor | None = None,
+                              beta: torch.Tensor | None = None, wq: torch.Tensor | None = None,
+                              sw: torch.Tensor | None = None, gamma_f: torch.Tensor | None = None,
+                              beta_f: torch.Tensor | None = None, stream=None):
+    """W [K, N] -> (Wq [N, K] E4M3 codes (uint8), sw [N], gamma / s or None, beta / s or None)."""
+    W = _mat(W, "W")
+    K, N = W.shape
+    _vec(s, K, "s")
+    _vec(gamma, K, "gamma")
+    _vec(beta, K, "beta")
+    dev = W.device
+    if wq is None:
+        wq = torch.empty(N, K, dtype=torch.uint8, device=dev)
+    if sw is None:
+        sw = torch.empty(N, dtype=torch.float32, device=dev)
+    gf = bf = None
+    if gamma is not None:
+        gf = gamma_f if gamma_f is not None else torch.empty(K, dtype=torch.float32, device=dev)
+    if beta is not None:
+        bf = beta_f if beta_f is not None else torch.empty(K, dtype=torch.float32, device=dev)
+    _check("sq_fold_quant_weights_fp8",
+           lib().sq_fold_quant_weights_fp8(_ptr(W), _dt(W), K, N, W.stride(0), _ptr(s), _ptr(gamma), _ptr(beta),
+                                           _ptr(wq), _ptr(sw), _ptr(gf), _ptr(bf), _stream(stream)))
+    return wq, sw, gf, bf
+
+
+def sq_ln_smooth_quant_fp8(x: torch.Tensor, gamma_f: torch.Tensor | None = None, beta_f: torch.Tensor | None = None,
+                           s: torch.Tensor | None = None, eps: float = 1e-5, xq: torch.Tensor | None = None,
+                           sx: torch.Tensor | None = None, stream=None):
+    """LayerNorm mode (gamma_f given) or plain mode (s given) -> (xq [M, K] E4M3 codes, sx [M])."""
+    x = _mat(x, "x")
+    M, K = x.shape
+    _vec(gamma_f, K, "gamma_f")
+    _vec(beta_f, K, "beta_f")
+    _vec(s, K, "s")
+    if xq is None:
+        xq = torch.empty(M, K, dtype=torch.uint8, device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check("sq_ln_smooth_quant_fp8",
+           lib().sq_ln_smooth_quant_fp8(_ptr(x), _dt(x), M, K, x.stride(0), _ptr(gamma_f), _ptr(beta_f), _ptr(s),
+                                        float(eps), _ptr(xq), _ptr(sx), _stream(stream)))
+    return xq, sx
+
+
+def sq_w8a8_gemm_fp8(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                     out_dtype: torch.dtype = torch.bfloat16, y: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = bf16((acc * sx[:, None]) * sw[None, :]) with acc = dec(xq) @ dec(wq)^T in fp32 (or f32 y)."""
+    if xq.dtype != torch.uint8 or wq.dtype != torch.uint8 or not xq.is_contiguous() or not wq.is_contiguous():
+        raise ValueError("xq and wq must be contiguous uint8 tensors of E4M3 codes")
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError("xq and wq disagree on K")
+    if y is None:
+        y = torch.empty(M, N, dtype=out_dtype, device=xq.device)
+    ydt = _ODT[y.dtype]
+    _vec(sx, M, "sx")
+    _vec(sw, N, "sw")
+    need = sq_w8a8_gemm_workspace_size(M, N, K)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=xq.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("sq_w8a8_gemm_fp8", lib().sq_w8a8_gemm_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
+                                                      y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))
     return y
 
 

@@ -26,6 +26,15 @@ cudaError_t launch_ln_smooth_quant_per_tensor(const void* x, bool bf16, int64_t 
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
                         int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
                         bool* ws_too_small);
+cudaError_t launch_fold_quant_fp8(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
+                                  const float* gamma, const float* beta, uint8_t* Wq, float* sw, float* gamma_f,
+                                  float* beta_f, cudaStream_t st);
+cudaError_t launch_ln_smooth_quant_fp8(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
+                                       const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                       uint8_t* xq, float* sx, cudaStream_t st);
+cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw, int64_t M,
+                            int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
+                            cudaStream_t st, bool* ws_too_small);
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 cudaError_t read_device_error(unsigned int* code, int clear, cudaStream_t st);
 
@@ -70,9 +79,79 @@ bool vec_ok(const float* p) { return p != nullptr && aligned16(p); }
 
 }  // namespace
 
+namespace {
+// Validation shared by the INT8 and FP8 folds; SQ_OK with *empty set means nothing to do.
+sq_status check_fold(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw, const float* s,
+                     const float* gamma, const float* beta, const void* Wq, const float* sw, const float* gamma_f,
+                     const float* beta_f, bool* empty) {
+  *empty = false;
+  if (K < 0 || N < 0) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_matrix(W, dt, K, N, ldw);
+  if (st != SQ_OK) return st;
+  if (K == 0 || N == 0) {
+    *empty = true;
+    return SQ_OK;
+  }
+  if (s == nullptr || !aligned4(s) || Wq == nullptr || sw == nullptr || !aligned4(sw)) return SQ_ERR_INVALID_ARG;
+  if ((gamma && !aligned4(gamma)) || (beta && !aligned4(beta)) || (gamma_f && !aligned4(gamma_f)) ||
+      (beta_f && !aligned4(beta_f)))
+    return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || !aligned16(Wq)) return SQ_ERR_ALIGNMENT;
+  if (K > SQ_MAX_K) return SQ_ERR_UNSUPPORTED;
+  return SQ_OK;
+}
+
+// Validation shared by the per-token INT8 and FP8 quantisers.
+sq_status check_row_quant(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
+                          const float* beta_f, const float* s, float eps, const void* xq, const float* sx,
+                          bool* empty) {
+  *empty = false;
+  if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  if ((gamma_f == nullptr) == (s == nullptr)) return SQ_ERR_INVALID_ARG;  // exactly one mode
+  if (gamma_f == nullptr && beta_f != nullptr) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_matrix(x, dt, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if ((gamma_f && !aligned16(gamma_f)) || (beta_f && !aligned16(beta_f)) || (s && !aligned16(s)))
+    return SQ_ERR_ALIGNMENT;
+  if (gamma_f && !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
+  if (M == 0) {
+    *empty = true;
+    return SQ_OK;
+  }
+  if (xq == nullptr || sx == nullptr || !aligned4(sx)) return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || !aligned16(xq)) return SQ_ERR_ALIGNMENT;
+  if (K > SQ_MAX_K_ROW || (dt == SQ_F32 && K > SQ_MAX_K_ROW / 2)) return SQ_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  return SQ_OK;
+}
+
+// Validation shared by the INT8 and FP8 GEMMs (the FP8 one has no int32 output).
+sq_status check_gemm(const void* xq, const float* sx, const void* wq, const float* sw, int64_t M, int64_t N,
+                     int64_t K, const void* y, sq_dtype ydt, int64_t ldy, const void* workspace, bool allow_i32,
+                     bool* empty) {
+  *empty = false;
+  if (M < 0 || N < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  if (ydt != SQ_BF16 && ydt != SQ_F32 && !(allow_i32 && ydt == SQ_I32)) return SQ_ERR_INVALID_ARG;
+  if (ldy < N) return SQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) {
+    *empty = true;
+    return SQ_OK;
+  }
+  if (!xq || !wq || !y) return SQ_ERR_INVALID_ARG;
+  if (ydt != SQ_I32 && (!sx || !sw || !aligned4(sx) || !aligned4(sw))) return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || !aligned16(xq) || !aligned16(wq)) return SQ_ERR_ALIGNMENT;
+  const uintptr_t e = ydt == SQ_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(y) % e != 0) return SQ_ERR_ALIGNMENT;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SQ_ERR_ALIGNMENT;
+  if (K > SQ_MAX_K) return SQ_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  return SQ_OK;
+}
+}  // namespace
+
 extern "C" {
 
-int sq_abi_version(void) { return 100; }
+int sq_abi_version(void) { return 101; }
 
 const char* sq_status_string(sq_status status) {
   switch (status) {
@@ -130,38 +209,54 @@ sq_status sq_smooth_factors(const float* ax, const float* aw, int64_t K, float a
   return cuda_status(sqh::launch_smooth_factors(ax, aw, K, alpha, s, as_stream(stream)));
 }
 
+sq_status sq_fold_quant_weights_fp8(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw, const float* s,
+                                    const float* gamma, const float* beta, uint8_t* Wq, float* sw, float* gamma_f,
+                                    float* beta_f, void* stream) {
+  bool empty = false;
+  const sq_status st = check_fold(W, dt, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, &empty);
+  if (st != SQ_OK || empty) return st;
+  return cuda_status(sqh::launch_fold_quant_fp8(W, dt == SQ_BF16, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f,
+                                                as_stream(stream)));
+}
+
+sq_status sq_ln_smooth_quant_fp8(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
+                                 const float* beta_f, const float* s, float eps, uint8_t* xq, float* sx,
+                                 void* stream) {
+  bool empty = false;
+  const sq_status st = check_row_quant(x, dt, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, &empty);
+  if (st != SQ_OK || empty) return st;
+  return cuda_status(sqh::launch_ln_smooth_quant_fp8(x, dt == SQ_BF16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx,
+                                                     as_stream(stream)));
+}
+
+sq_status sq_w8a8_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw, int64_t M,
+                           int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  bool empty = false;
+  const sq_status st = check_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, workspace, false, &empty);
+  if (st != SQ_OK || empty) return st;
+  bool ws_small = false;
+  cudaError_t err = sqh::launch_gemm_fp8(xq, sx, wq, sw, M, N, K, y, (int)ydt, ldy, workspace, ws_bytes,
+                                         as_stream(stream), &ws_small);
+  if (ws_small) return SQ_ERR_WORKSPACE;
+  return cuda_status(err);
+}
+
 sq_status sq_fold_quant_weights(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw, const float* s,
                                 const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
                                 float* beta_f, void* stream) {
-  if (K < 0 || N < 0) return SQ_ERR_INVALID_ARG;
-  sq_status st = check_matrix(W, dt, K, N, ldw);
-  if (st != SQ_OK) return st;
-  if (K == 0 || N == 0) return SQ_OK;
-  if (s == nullptr || !aligned4(s) || Wq == nullptr || sw == nullptr || !aligned4(sw)) return SQ_ERR_INVALID_ARG;
-  if ((gamma && !aligned4(gamma)) || (beta && !aligned4(beta)) || (gamma_f && !aligned4(gamma_f)) ||
-      (beta_f && !aligned4(beta_f)))
-    return SQ_ERR_INVALID_ARG;
-  if (K % 16 != 0 || !aligned16(Wq)) return SQ_ERR_ALIGNMENT;
-  if (K > SQ_MAX_K) return SQ_ERR_UNSUPPORTED;
+  bool empty = false;
+  const sq_status st = check_fold(W, dt, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, &empty);
+  if (st != SQ_OK || empty) return st;
   return cuda_status(sqh::launch_fold_quant(W, dt == SQ_BF16, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f,
                                             as_stream(stream)));
 }
 
 sq_status sq_ln_smooth_quant(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                              const float* beta_f, const float* s, float eps, int8_t* xq, float* sx, void* stream) {
-  if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
-  if ((gamma_f == nullptr) == (s == nullptr)) return SQ_ERR_INVALID_ARG;  // exactly one mode
-  if (gamma_f == nullptr && beta_f != nullptr) return SQ_ERR_INVALID_ARG;
-  sq_status st = check_matrix(x, dt, M, K, ldx);
-  if (st != SQ_OK) return st;
-  if ((gamma_f && !aligned16(gamma_f)) || (beta_f && !aligned16(beta_f)) || (s && !aligned16(s)))
-    return SQ_ERR_ALIGNMENT;
-  if (gamma_f && !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
-  if (M == 0) return SQ_OK;
-  if (xq == nullptr || sx == nullptr || !aligned4(sx)) return SQ_ERR_INVALID_ARG;
-  if (K % 16 != 0 || !aligned16(xq)) return SQ_ERR_ALIGNMENT;
-  if (K > SQ_MAX_K_ROW || (dt == SQ_F32 && K > SQ_MAX_K_ROW / 2)) return SQ_ERR_UNSUPPORTED;
-  if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  bool empty = false;
+  const sq_status st = check_row_quant(x, dt, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, &empty);
+  if (st != SQ_OK || empty) return st;
   return cuda_status(
       sqh::launch_ln_smooth_quant(x, dt == SQ_BF16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, as_stream(stream)));
 }
@@ -171,19 +266,9 @@ sq_status sq_ln_smooth_quant_per_tensor(const void* x, sq_dtype dt, int64_t M, i
                                         int static_scale, float* scale, int8_t* xq, float* sx, void* stream) {
   if (static_scale != 0 && static_scale != 1) return SQ_ERR_INVALID_ARG;
   if (scale == nullptr || !aligned4(scale)) return SQ_ERR_INVALID_ARG;
-  if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
-  if ((gamma_f == nullptr) == (s == nullptr)) return SQ_ERR_INVALID_ARG;  // exactly one mode
-  if (gamma_f == nullptr && beta_f != nullptr) return SQ_ERR_INVALID_ARG;
-  sq_status st = check_matrix(x, dt, M, K, ldx);
-  if (st != SQ_OK) return st;
-  if ((gamma_f && !aligned16(gamma_f)) || (beta_f && !aligned16(beta_f)) || (s && !aligned16(s)))
-    return SQ_ERR_ALIGNMENT;
-  if (gamma_f && !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
-  if (M == 0) return SQ_OK;
-  if (xq == nullptr || sx == nullptr || !aligned4(sx)) return SQ_ERR_INVALID_ARG;
-  if (K % 16 != 0 || !aligned16(xq)) return SQ_ERR_ALIGNMENT;
-  if (K > SQ_MAX_K_ROW || (dt == SQ_F32 && K > SQ_MAX_K_ROW / 2)) return SQ_ERR_UNSUPPORTED;
-  if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  bool empty = false;
+  const sq_status st = check_row_quant(x, dt, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, &empty);
+  if (st != SQ_OK || empty) return st;
   return cuda_status(sqh::launch_ln_smooth_quant_per_tensor(x, dt == SQ_BF16, M, K, ldx, gamma_f, beta_f, s, eps,
                                                             static_scale, scale, xq, sx, as_stream(stream)));
 }
@@ -196,18 +281,9 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
                        int64_t K, void* y, sq_dtype ydt, int64_t ldy, void* workspace, size_t ws_bytes, void* stream) {
-  if (M < 0 || N < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
-  if (ydt != SQ_BF16 && ydt != SQ_F32 && ydt != SQ_I32) return SQ_ERR_INVALID_ARG;
-  if (ldy < N) return SQ_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return SQ_OK;
-  if (!xq || !wq || !y) return SQ_ERR_INVALID_ARG;
-  if (ydt != SQ_I32 && (!sx || !sw || !aligned4(sx) || !aligned4(sw))) return SQ_ERR_INVALID_ARG;
-  if (K % 16 != 0 || !aligned16(xq) || !aligned16(wq)) return SQ_ERR_ALIGNMENT;
-  const uintptr_t e = ydt == SQ_BF16 ? 2 : 4;
-  if (reinterpret_cast<uintptr_t>(y) % e != 0) return SQ_ERR_ALIGNMENT;
-  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SQ_ERR_ALIGNMENT;
-  if (K > SQ_MAX_K) return SQ_ERR_UNSUPPORTED;
-  if (M > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  bool empty = false;
+  const sq_status st = check_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, workspace, true, &empty);
+  if (st != SQ_OK || empty) return st;
   bool ws_small = false;
   cudaError_t err = sqh::launch_gemm(xq, sx, wq, sw, M, N, K, y, (int)ydt, ldy, workspace, ws_bytes,
                                      as_stream(stream), &ws_small);

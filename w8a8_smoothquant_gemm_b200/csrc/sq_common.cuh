@@ -124,6 +124,59 @@ __device__ __forceinline__ uint2 pack8_codes(const float* y, const SharedDivisor
   return make_uint2(pack4_low_bytes(c[0], c[1], c[2], c[3]), pack4_low_bytes(c[4], c[5], c[6], c[7]));
 }
 
+// ---------------------------------------------------------------------------- FP8 codes
+// The FP8 variant of the method uses E4M3 codes (OCP 8-bit floating point, OFP8: bias 7,
+// 3 mantissa bits, largest finite 448) with scale = max|.| / 448; the code of v is E4M3 of
+// the correctly rounded quotient RN(v / scale), nearest even, saturating.
+
+// E4M3 codes of four binary32 values, first argument in the low byte (the PTX conversion
+// puts its first source operand in the upper byte of each pair).
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
+// E4M3 code (byte value) of v with a scale: E4M3 of the correctly rounded RN(v / scale);
+// scale 0 -> +0.
+__device__ __forceinline__ int e4m3_code(float v, float scale) {
+  if (scale == 0.0f) return 0;
+  return (int)(e4m3x4(__fdiv_rn(v, scale), 0.0f, 0.0f, 0.0f) & 0xffu);
+}
+
+// The quotient with the dividend's sign: Markstein's correction step turns RN(-0 / b) = -0
+// into +0, which E4M3 (unlike an integer code) tells apart.
+__device__ __forceinline__ float with_sign_of(float q, float v) { return copysignf(q, v); }
+
+// E4M3 codes of 8 values (one chunk) with a shared scale; a zero scale (all-zero row or
+// column) gives +0 codes.
+template <bool FAST>
+__device__ __forceinline__ uint2 pack8_e4m3(const float* y, const SharedDivisor& d) {
+  if (d.fast && d.y == 0.0f) return make_uint2(0u, 0u);  // zero scale
+  float q[8];
+  if (FAST) {
+    const float2 rc = make_float2(d.y, d.y), nb = make_float2(-d.b, -d.b);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float2 a = make_float2(y[e], y[e + 1]);
+      const float2 q0 = __fmul2_rn(a, rc);
+      const float2 r = __ffma2_rn(q0, nb, a);
+      const float2 qq = __ffma2_rn(r, rc, q0);
+      q[e] = with_sign_of(qq.x, y[e]);
+      q[e + 1] = with_sign_of(qq.y, y[e + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q[e] = d.div(y[e]);  // correctly rounded division keeps the sign
+  }
+  return make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+}
+
 // Writes the codes of NCH chunks (chunk m of this thread at c = t + T m) of one row.
 template <int T, int NCH>
 __device__ __forceinline__ void store_row_codes(const float* v, int t, int nchunks, float scale, bool clamp,

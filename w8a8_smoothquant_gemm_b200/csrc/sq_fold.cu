@@ -54,7 +54,7 @@ __device__ __forceinline__ void load8(const char* p, float f[8]) {
 // Block: 256 threads = (CW/8 column groups of 8) x (256 / (CW/8) row lanes).
 // Pass-2 tile: TJ rows (j) x CW columns (k); codes staged transposed in shared memory as
 // [CW][TJ + 16] bytes, then written as CW rows of TJ contiguous bytes of Wq.
-template <bool BF16, int CW>
+template <bool BF16, int CW, bool F8>
 __global__ void __launch_bounds__(256)
 fold_quant_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_bytes,
                   const float* __restrict__ s, const float* __restrict__ gamma, const float* __restrict__ beta,
@@ -118,7 +118,7 @@ fold_quant_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_
     if (threadIdx.x < CW) {
       float v = red[0][threadIdx.x];
       for (int r = 1; r < NR; ++r) v = fmaxf(v, red[r][threadIdx.x]);
-      const float sc = __fdiv_rn(v, 127.0f);
+      const float sc = __fdiv_rn(v, F8 ? 448.0f : 127.0f);
       scale_s[threadIdx.x] = sc;
       if (k0 + threadIdx.x < N) sw[k0 + threadIdx.x] = sc;
     }
@@ -137,7 +137,7 @@ fold_quant_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_
           load8<BF16>(W + j * ldw_bytes + kc * ELT, f);
           const float sj = __ldg(s + j);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) q[e] = quant_code(__fmul_rn(sj, f[e]), sc[e]);
+          for (int e = 0; e < 8; ++e) q[e] = F8 ? e4m3_code(__fmul_rn(sj, f[e]), sc[e]) : quant_code(__fmul_rn(sj, f[e]), sc[e]);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) stage[g * 8 + e][jj] = (int8_t)q[e];
@@ -172,6 +172,11 @@ __device__ __forceinline__ void fold_codes_16x4(const uint16_t* tile, const floa
                                                 const SharedDivisor& d0, const SharedDivisor& d1,
                                                 const SharedDivisor& d2, const SharedDivisor& d3,
                                                 uint32_t (&words)[4][4]) {
+  // two adjacent columns per packed binary32 pair, each with its own scale; each half
+  // rounds as the scalar operation would
+  const float2 rc01 = make_float2(d0.y, d1.y), rc23 = make_float2(d2.y, d3.y);
+  const float2 nb01 = make_float2(-d0.b, -d1.b), nb23 = make_float2(-d2.b, -d3.b);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
 #pragma unroll
   for (int g4 = 0; g4 < 4; ++g4) {
     uint32_t b[4][4];
@@ -180,16 +185,22 @@ __device__ __forceinline__ void fold_codes_16x4(const uint16_t* tile, const floa
       const int j = jl + g4 * 4 + r;
       const uint2 w = *reinterpret_cast<const uint2*>(tile + j * cw + kq);
       const float sj = s_rows[j];
+      const float2 y01 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.x), bf16hi(w.x)));
+      const float2 y23 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.y), bf16hi(w.y)));
       if (FAST) {
-        b[0][r] = code_bits_fast(__fmul_rn(sj, bf16lo(w.x)), d0);
-        b[1][r] = code_bits_fast(__fmul_rn(sj, bf16hi(w.x)), d1);
-        b[2][r] = code_bits_fast(__fmul_rn(sj, bf16lo(w.y)), d2);
-        b[3][r] = code_bits_fast(__fmul_rn(sj, bf16hi(w.y)), d3);
+        const float2 q01 = __fmul2_rn(y01, rc01), q23 = __fmul2_rn(y23, rc23);
+        const float2 e01 = __ffma2_rn(q01, nb01, y01), e23 = __ffma2_rn(q23, nb23, y23);
+        const float2 t01 = __fadd2_rn(__ffma2_rn(e01, rc01, q01), magic);
+        const float2 t23 = __fadd2_rn(__ffma2_rn(e23, rc23, q23), magic);
+        b[0][r] = __float_as_uint(t01.x);
+        b[1][r] = __float_as_uint(t01.y);
+        b[2][r] = __float_as_uint(t23.x);
+        b[3][r] = __float_as_uint(t23.y);
       } else {
-        b[0][r] = code_bits(__fmul_rn(sj, bf16lo(w.x)), d0);
-        b[1][r] = code_bits(__fmul_rn(sj, bf16hi(w.x)), d1);
-        b[2][r] = code_bits(__fmul_rn(sj, bf16lo(w.y)), d2);
-        b[3][r] = code_bits(__fmul_rn(sj, bf16hi(w.y)), d3);
+        b[0][r] = code_bits(y01.x, d0);
+        b[1][r] = code_bits(y01.y, d1);
+        b[2][r] = code_bits(y23.x, d2);
+        b[3][r] = code_bits(y23.y, d3);
       }
     }
 #pragma unroll
@@ -197,10 +208,86 @@ __device__ __forceinline__ void fold_codes_16x4(const uint16_t* tile, const floa
   }
 }
 
+// E4M3 codes of a 16-row x 4-column block (the FP8 variant): the quotients of
+// fold_codes_16x4 with the dividend's sign kept on zero results (Markstein's correction
+// turns RN(-0 / b) into +0), converted with saturation; a zero scale gives +0 codes.
+// FAST: every scale nonzero and in Markstein's range.
+template <bool FAST>
+__device__ __forceinline__ void fold_codes_16x4_e4m3(const uint16_t* tile, const float* s_rows, int cw, int jl, int kq,
+                                                     const SharedDivisor& d0, const SharedDivisor& d1,
+                                                     const SharedDivisor& d2, const SharedDivisor& d3,
+                                                     uint32_t (&words)[4][4]) {
+  const float2 rc01 = make_float2(d0.y, d1.y), rc23 = make_float2(d2.y, d3.y);
+  const float2 nb01 = make_float2(-d0.b, -d1.b), nb23 = make_float2(-d2.b, -d3.b);
+  const SharedDivisor* dv[4] = {&d0, &d1, &d2, &d3};
+#pragma unroll
+  for (int g4 = 0; g4 < 4; ++g4) {
+    float q[4][4];  // [column][row]
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = jl + g4 * 4 + r;
+      const uint2 w = *reinterpret_cast<const uint2*>(tile + j * cw + kq);
+      const float sj = s_rows[j];
+      const float2 y01 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.x), bf16hi(w.x)));
+      const float2 y23 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.y), bf16hi(w.y)));
+      if (FAST) {
+        const float2 q01 = __fmul2_rn(y01, rc01), q23 = __fmul2_rn(y23, rc23);
+        const float2 t01 = __ffma2_rn(__ffma2_rn(q01, nb01, y01), rc01, q01);
+        const float2 t23 = __ffma2_rn(__ffma2_rn(q23, nb23, y23), rc23, q23);
+        q[0][r] = with_sign_of(t01.x, y01.x);
+        q[1][r] = with_sign_of(t01.y, y01.y);
+        q[2][r] = with_sign_of(t23.x, y23.x);
+        q[3][r] = with_sign_of(t23.y, y23.y);
+      } else {
+        const float y[4] = {y01.x, y01.y, y23.x, y23.y};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          q[c][r] = (dv[c]->fast && dv[c]->y == 0.0f) ? 0.0f : with_sign_of(dv[c]->div(y[c]), y[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) words[c][g4] = e4m3x4(q[c][0], q[c][1], q[c][2], q[c][3]);
+  }
+}
+
+// Codes of this CTA's rows of the strip at column k0 from the staged tile, with the
+// strip's scales, written to Wq transposed: item = (4 adjacent columns, 16 consecutive
+// rows); each item reads 16 x 8 bytes of shared memory and writes 16 codes to each of 4
+// rows of Wq.  F8: E4M3 codes (the FP8 variant).
+template <int CW, bool F8>
+__device__ __forceinline__ void fold_write_codes(const uint16_t* tile, const float* s_rows, const float* scale,
+                                                 int64_t K, int64_t N, int RK, int64_t j0, int64_t k0,
+                                                 int8_t* __restrict__ Wq) {
+  const int items = (CW / 4) * (RK / 16);
+  for (int i = threadIdx.x; i < items; i += 256) {
+    const int kq = (i % (CW / 4)) * 4, jl = (i / (CW / 4)) * 16;
+    if (j0 + jl >= K) continue;  // K % 16 == 0: a 16-row block is all in or all out
+    const SharedDivisor d0(scale[kq]), d1(scale[kq + 1]), d2(scale[kq + 2]), d3(scale[kq + 3]);
+    uint32_t words[4][4];
+    const bool fast = d0.fast && d1.fast && d2.fast && d3.fast;
+    if (F8) {
+      if (fast && d0.y != 0.0f && d1.y != 0.0f && d2.y != 0.0f && d3.y != 0.0f)
+        fold_codes_16x4_e4m3<true>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
+      else
+        fold_codes_16x4_e4m3<false>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
+    } else if (fast) {
+      fold_codes_16x4<true>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
+    } else {
+      fold_codes_16x4<false>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t k = k0 + kq + c;
+      if (k < N)
+        *reinterpret_cast<uint4*>(Wq + k * K + j0 + jl) = make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
+    }
+  }
+}
+
 constexpr int FOLD_MAX_CLUSTER = 16;
 constexpr int FOLD_MAX_PIECES = 64;  // RK <= 4096 rows per CTA
 
-template <int CW>
+template <int CW, bool F8>
 __global__ void __launch_bounds__(256)
 fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t N, int RK, int C,
                     const float* __restrict__ s, const float* __restrict__ gamma, const float* __restrict__ beta,
@@ -257,11 +344,15 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
       if (!mbar_wait(smem_u32(&bars[p]), 0)) atomicOr(err, ERR_FOLD_TMA_WAIT);
       for (int j = p * 64 + rl; j < p * 64 + 64; j += G) {
         const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
-        const float sj = s_rows[j];
-        float f[8];
-        unpack8_bf16(w, f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(sj, f[e])));
+        const float2 sj = make_float2(s_rows[j], s_rows[j]);
+        const float2 y0 = __fmul2_rn(sj, make_float2(bf16lo(w.x), bf16hi(w.x)));
+        const float2 y1 = __fmul2_rn(sj, make_float2(bf16lo(w.y), bf16hi(w.y)));
+        const float2 y2 = __fmul2_rn(sj, make_float2(bf16lo(w.z), bf16hi(w.z)));
+        const float2 y3 = __fmul2_rn(sj, make_float2(bf16lo(w.w), bf16hi(w.w)));
+        m[0] = fmaxf(m[0], fabsf(y0.x)); m[1] = fmaxf(m[1], fabsf(y0.y));
+        m[2] = fmaxf(m[2], fabsf(y1.x)); m[3] = fmaxf(m[3], fabsf(y1.y));
+        m[4] = fmaxf(m[4], fabsf(y2.x)); m[5] = fmaxf(m[5], fabsf(y2.y));
+        m[6] = fmaxf(m[6], fabsf(y3.x)); m[7] = fmaxf(m[7], fabsf(y3.y));
       }
     }
 #pragma unroll
@@ -277,31 +368,130 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
   if (tid < CW) {
     float m = 0.0f;
     for (int r = 0; r < C; ++r) m = fmaxf(m, part[r][tid]);
-    const float sc = __fdiv_rn(m, 127.0f);
+    const float sc = __fdiv_rn(m, F8 ? 448.0f : 127.0f);
     scale[tid] = sc;
     if (crank == 0 && k0 + tid < N) sw[k0 + tid] = sc;
   }
   __syncthreads();
 
-  // ---- codes, transposed: item = (4 adjacent columns, 16 consecutive rows); each item
-  // reads 16 x 8 bytes of shared memory and writes 16 codes to each of 4 rows of Wq.
-  const int items = (CW / 4) * (RK / 16);
-  for (int it = tid; it < items; it += 256) {
-    const int kq = (it % (CW / 4)) * 4, jl = (it / (CW / 4)) * 16;
-    if (j0 + jl >= K) continue;  // K % 16 == 0: a 16-row block is all in or all out
-    const SharedDivisor d0(scale[kq]), d1(scale[kq + 1]), d2(scale[kq + 2]), d3(scale[kq + 3]);
-    uint32_t words[4][4];
-    if (d0.fast && d1.fast && d2.fast && d3.fast)
-      fold_codes_16x4<true>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
-    else
-      fold_codes_16x4<false>(tile, s_rows, CW, jl, kq, d0, d1, d2, d3, words);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int64_t k = k0 + kq + c;
-      if (k < N)
-        *reinterpret_cast<uint4*>(Wq + k * K + j0 + jl) = make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
-    }
+  // ---- codes, transposed
+  fold_write_codes<CW, F8>(tile, s_rows, scale, K, N, RK, j0, k0, Wq);
+}
+
+// Fold for tall blocks (large K, where one strip's block of a CTA takes most of the shared
+// memory): clusters stay resident and walk over strips (strip = cluster, cluster +
+// clusters, ...), with two tile buffers per CTA.  Iteration i: column max of strip i,
+// partials pushed to every peer, cluster-barrier arrive | codes of strip i-1 (its scales
+// are known) | cluster-barrier wait, scales of strip i | load of strip i+1 into the buffer
+// strip i-1 used.  The cluster barrier's latency is covered by the previous strip's codes.
+template <int CW, bool F8>
+__global__ void __launch_bounds__(256)
+fold_stream_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t N, int RK, int C,
+                    const float* __restrict__ s, const float* __restrict__ gamma, const float* __restrict__ beta,
+                    int8_t* __restrict__ Wq, float* __restrict__ sw, float* __restrict__ gamma_f,
+                    float* __restrict__ beta_f, unsigned int* err) {
+  constexpr int G = 256 / (CW / 8);  // row lanes of the max pass (8 columns per thread)
+  constexpr int NBUF = 2;
+  extern __shared__ uint8_t smem_raw[];
+  // TMA destinations want 128-byte alignment: round the dynamic base up (128 bytes of slack)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const size_t tile_bytes = (size_t)RK * CW * 2;
+  float* s_rows = reinterpret_cast<float*>(smem + NBUF * tile_bytes);  // [RK]
+  __shared__ float red[G][CW + 1];
+  __shared__ float part[2][FOLD_MAX_CLUSTER][CW];  // partial maxima of every CTA, by strip parity
+  __shared__ float scale[2][CW];
+  __shared__ __align__(8) uint64_t bars[NBUF];
+
+  const int tid = threadIdx.x;
+  const uint32_t crank = cluster_ctarank();
+  const int64_t clusters = gridDim.x / C;
+  const int64_t strips = (N + CW - 1) / CW;
+  const int64_t j0 = (int64_t)crank * RK;
+  const int pieces = RK / 64;
+
+  for (int64_t j = (int64_t)blockIdx.x * 256 + tid; j < K; j += (int64_t)gridDim.x * 256) {
+    const float sj = s[j];
+    if (gamma && gamma_f) gamma_f[j] = __fdiv_rn(gamma[j], sj);
+    if (beta && beta_f) beta_f[j] = __fdiv_rn(beta[j], sj);
   }
+
+  if (tid == 0) {
+    for (int b = 0; b < NBUF; ++b) mbar_init(smem_u32(&bars[b]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = tid; i < RK; i += 256) s_rows[i] = (j0 + i < K) ? __ldg(s + j0 + i) : 0.0f;
+  __syncthreads();
+
+  // one thread: the RK x CW block of strip number `n` of this cluster into its buffer (after
+  // a barrier that ended every generic read of that buffer)
+  const int64_t first = blockIdx.x / C;
+  auto issue = [&](int64_t n) {
+    const int buf = (int)(n % NBUF);
+    const uint32_t b = smem_u32(&bars[buf]);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(b, (uint32_t)tile_bytes);
+    const int64_t strip = first + n * clusters;
+    for (int p = 0; p < pieces; ++p)
+      tma_load_2d(smem_u32(smem + buf * tile_bytes + (size_t)p * 64 * CW * 2), &wmap, b, (int)(strip * CW),
+                  (int)(j0 + p * 64));
+  };
+  const int64_t count = first < strips ? (strips - first + clusters - 1) / clusters : 0;  // strips of this cluster
+  if (tid == 0 && count > 0) issue(0);
+
+  for (int64_t n = 0; n < count; ++n) {
+    const int buf = (int)(n % NBUF), par = (int)(n & 1);
+    const uint16_t* tile = reinterpret_cast<const uint16_t*>(smem + buf * tile_bytes);
+    if (!mbar_wait(smem_u32(&bars[buf]), (uint32_t)((n / NBUF) & 1))) atomicOr(err, ERR_FOLD_TMA_WAIT);
+
+    // ---- partial column max of |s_j W_jk| over this CTA's rows: thread = 8 columns x rows
+    // rl, rl + G, ...
+    {
+      const int cg = tid % (CW / 8), rl = tid / (CW / 8);
+      float m[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = 0.0f;
+#pragma unroll 4
+      for (int j = rl; j < RK; j += G) {
+        const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
+        const float2 sj = make_float2(s_rows[j], s_rows[j]);
+        const float2 y0 = __fmul2_rn(sj, make_float2(bf16lo(w.x), bf16hi(w.x)));
+        const float2 y1 = __fmul2_rn(sj, make_float2(bf16lo(w.y), bf16hi(w.y)));
+        const float2 y2 = __fmul2_rn(sj, make_float2(bf16lo(w.z), bf16hi(w.z)));
+        const float2 y3 = __fmul2_rn(sj, make_float2(bf16lo(w.w), bf16hi(w.w)));
+        m[0] = fmaxf(m[0], fabsf(y0.x)); m[1] = fmaxf(m[1], fabsf(y0.y));
+        m[2] = fmaxf(m[2], fabsf(y1.x)); m[3] = fmaxf(m[3], fabsf(y1.y));
+        m[4] = fmaxf(m[4], fabsf(y2.x)); m[5] = fmaxf(m[5], fabsf(y2.y));
+        m[6] = fmaxf(m[6], fabsf(y3.x)); m[7] = fmaxf(m[7], fabsf(y3.y));
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
+    }
+    __syncthreads();
+    if (tid < CW) {
+      float m = red[0][tid];
+      for (int g = 1; g < G; ++g) m = fmaxf(m, red[g][tid]);
+      for (int r = 0; r < C; ++r) st_dsmem_f32(&part[par][crank][tid], (uint32_t)r, m);  // into every CTA
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    // the previous strip's codes while the partials of this one are in flight
+    if (n > 0)
+      fold_write_codes<CW, F8>(reinterpret_cast<const uint16_t*>(smem + ((n - 1) % NBUF) * tile_bytes), s_rows,
+                           scale[par ^ 1], K, N, RK, j0, (first + (n - 1) * clusters) * CW, Wq);
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // every partial of strip n is here
+    if (tid < CW) {
+      float m = 0.0f;
+      for (int r = 0; r < C; ++r) m = fmaxf(m, part[par][r][tid]);
+      const float sc = __fdiv_rn(m, F8 ? 448.0f : 127.0f);
+      scale[par][tid] = sc;
+      const int64_t k0 = (first + n * clusters) * CW;
+      if (crank == 0 && k0 + tid < N) sw[k0 + tid] = sc;
+    }
+    __syncthreads();  // scales visible; red and the previous strip's buffer free
+    if (tid == 0 && n + 1 < count) issue(n + 1);  // strip n-1's buffer is free now
+  }
+  if (count > 0)
+    fold_write_codes<CW, F8>(reinterpret_cast<const uint16_t*>(smem + ((count - 1) % NBUF) * tile_bytes), s_rows,
+                         scale[(count - 1) & 1], K, N, RK, j0, (first + (count - 1) * clusters) * CW, Wq);
 }
 
 }  // namespace sqk
@@ -315,7 +505,7 @@ cudaError_t launch_smooth_factors(const float* ax, const float* aw, int64_t K, f
   return cudaGetLastError();
 }
 
-template <bool BF16, int CW>
+template <bool BF16, int CW, bool F8>
 static cudaError_t launch_fold_t(const void* W, int64_t K, int64_t N, int64_t ldw, const float* s, const float* gamma,
                                  const float* beta, int8_t* Wq, float* sw, float* gamma_f, float* beta_f,
                                  cudaStream_t st) {
@@ -331,19 +521,19 @@ static cudaError_t launch_fold_t(const void* W, int64_t K, int64_t N, int64_t ld
   int64_t grid = std::min<int64_t>(nstrips, std::max<int64_t>(std::min<int64_t>(fit, (int64_t)num_sms() * 4),
                                                               (int64_t)num_sms()));
   grid = std::max<int64_t>(grid, 1);
-  sqk::fold_quant_kernel<BF16, CW><<<(unsigned)grid, 256, 0, st>>>((const char*)W, K, N, ldw * elt, s, gamma, beta,
+  sqk::fold_quant_kernel<BF16, CW, F8><<<(unsigned)grid, 256, 0, st>>>((const char*)W, K, N, ldw * elt, s, gamma, beta,
                                                                    Wq, sw, gamma_f, beta_f);
   return cudaGetLastError();
 }
 
-template <int CW>
+template <int CW, bool F8>
 static cudaError_t launch_fold_cluster_t(const void* W, int64_t K, int64_t N, int64_t ldw, int C, int RK,
                                          const float* s, const float* gamma, const float* beta, int8_t* Wq,
                                          float* sw, float* gamma_f, float* beta_f, cudaStream_t st) {
   CUtensorMap map;
   if (!make_tmap_2d(&map, true, W, N, K, ldw * 2, CW, 64, false)) return cudaErrorInvalidValue;
   const size_t smem = 128 + (size_t)RK * CW * 2 + (size_t)RK * 4;
-  auto kern = sqk::fold_cluster_kernel<CW>;
+  auto kern = sqk::fold_cluster_kernel<CW, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (C > 8) {
@@ -366,6 +556,44 @@ static cudaError_t launch_fold_cluster_t(const void* W, int64_t K, int64_t N, in
   return cudaLaunchKernelEx(&cfg, kern, map, K, N, RK, C, s, gamma, beta, Wq, sw, gamma_f, beta_f, error_word_ptr());
 }
 
+static size_t fold_stream_smem(int64_t rk, int cw) { return 128 + 2 * (size_t)rk * cw * 2 + (size_t)rk * 4; }
+
+template <int CW, bool F8>
+static cudaError_t launch_fold_stream_t(const void* W, int64_t K, int64_t N, int64_t ldw, int C, int RK,
+                                         const float* s, const float* gamma, const float* beta, int8_t* Wq,
+                                         float* sw, float* gamma_f, float* beta_f, cudaStream_t st) {
+  CUtensorMap map;
+  if (!make_tmap_2d(&map, true, W, N, K, ldw * 2, CW, 64, false)) return cudaErrorInvalidValue;
+  const size_t smem = fold_stream_smem(RK, CW);
+  auto kern = sqk::fold_stream_kernel<CW, F8>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t strips = (N + CW - 1) / CW;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // as many clusters as are resident at once (each walks over strips), no more than strips
+  cfg.gridDim = dim3((unsigned)C);
+  int resident = 0;
+  e = cudaOccupancyMaxActiveClusters(&resident, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(strips, resident));
+  cfg.gridDim = dim3((unsigned)(clusters * C));
+  return cudaLaunchKernelEx(&cfg, kern, map, K, N, RK, C, s, gamma, beta, Wq, sw, gamma_f, beta_f, error_word_ptr());
+}
+
 // Cluster shape of the single-pass fold: C CTAs share a strip (at least 256 rows each, at
 // most 16), and the strip is the widest CW whose per-CTA block fits `budget` bytes of
 // shared memory.
@@ -383,26 +611,62 @@ static bool fold_cluster_shape(int64_t K, size_t budget, int* cw, int* c, int* r
   return false;
 }
 
-cudaError_t launch_fold_quant(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
+// Shape of the streaming fold (blocks taller than the one-shot fold's budget): the widest
+// CW whose two RK x CW buffers and factors fit 212 KB.
+static bool fold_stream_shape(int64_t K, int* cw, int* c, int* rk) {
+  const int cl = (int)std::min<int64_t>(16, std::max<int64_t>(1, (K + 255) / 256));
+  const int64_t rows = ((K + cl - 1) / cl + 63) / 64 * 64;
+  for (int w : {64, 32, 16})
+    if (fold_stream_smem(rows, w) <= 212 * 1024) {
+      *cw = w;
+      *c = cl;
+      *rk = (int)rows;
+      return true;
+    }
+  return false;
+}
+
+template <bool F8>
+static cudaError_t launch_fold_any(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
                               const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
                               float* beta_f, cudaStream_t st) {
   int cw = 0, cl = 0, rk = 0;
-  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 &&
-      (fold_cluster_shape(K, 72 * 1024, &cw, &cl, &rk) || fold_cluster_shape(K, 200 * 1024, &cw, &cl, &rk))) {
+  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_cluster_shape(K, 72 * 1024, &cw, &cl, &rk)) {
     switch (cw) {
-      case 64: return launch_fold_cluster_t<64>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-      case 32: return launch_fold_cluster_t<32>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-      default: return launch_fold_cluster_t<16>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      case 64: return launch_fold_cluster_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      case 32: return launch_fold_cluster_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      default: return launch_fold_cluster_t<16, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+    }
+  }
+  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_stream_shape(K, &cw, &cl, &rk)) {
+    switch (cw) {
+      case 64: return launch_fold_stream_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      case 32: return launch_fold_stream_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      default: return launch_fold_stream_t<16, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
     }
   }
   // narrower strips when there are few output channels, so every SM gets work
   const int64_t sms = num_sms();
   const int strip = (N / 32 >= 2 * sms) ? 32 : 16;
   if (bf16)
-    return strip == 32 ? launch_fold_t<true, 32>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
-                    : launch_fold_t<true, 16>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-  return strip == 32 ? launch_fold_t<false, 32>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
-                  : launch_fold_t<false, 16>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+    return strip == 32 ? launch_fold_t<true, 32, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
+                    : launch_fold_t<true, 16, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+  return strip == 32 ? launch_fold_t<false, 32, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
+                  : launch_fold_t<false, 16, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+}
+
+cudaError_t launch_fold_quant(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
+                              const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
+                              float* beta_f, cudaStream_t st) {
+  return launch_fold_any<false>(W, bf16, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+}
+
+// FP8 variant: E4M3 codes, sw = column max / 448.
+cudaError_t launch_fold_quant_fp8(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
+                                  const float* gamma, const float* beta, uint8_t* Wq, float* sw, float* gamma_f,
+                                  float* beta_f, cudaStream_t st) {
+  return launch_fold_any<true>(W, bf16, K, N, ldw, s, gamma, beta, reinterpret_cast<int8_t*>(Wq), sw, gamma_f,
+                               beta_f, st);
 }
 
 }  // namespace sqh

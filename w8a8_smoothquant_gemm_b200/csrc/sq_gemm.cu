@@ -1,7 +1,8 @@
 // sq_gemm.cu -- INT8 x INT8 -> int32 GEMM with the SmoothQuant dequant epilogue on the
-// 5th-generation (tcgen05) tensor cores of sm_100a.
+// 5th-generation (tcgen05) tensor cores of sm_100a, and its FP8 (E4M3 x E4M3 -> fp32)
+// variant on the same pipeline (tcgen05.mma kind::f8f6f4).
 //
-//   acc[m, n] = sum_j xq[m, j] * wq[n, j]            exact int32
+//   acc[m, n] = sum_j xq[m, j] * wq[n, j]            exact int32 (FP8: fp32 accumulation)
 //   y[m, n]   = bf16_rne(((float)acc * sx[m]) * sw[n])
 //
 // "4.2 W8A8 量化与 SmoothQuant" (intro, sec. 6): W8A8 lets the whole GEMM run on the INT8
@@ -28,7 +29,6 @@
 #include <cuda.h>
 
 #include <algorithm>
-#include <cstdlib>
 
 #include "sq_ptx.cuh"
 
@@ -94,12 +94,27 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
       : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, int8 -> int32; CG = 2 spans the CTA pair
-// (M = 256, each CTA supplies 128 rows of A and half of B from the same smem offsets).
-template <int CG>
-__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  if (CG == 1)
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, int8 -> int32 (F8: E4M3 -> fp32); CG = 2
+// spans the CTA pair (M = 256, each CTA supplies 128 rows of A and half of B from the same
+// smem offsets).
+template <int CG, bool F8>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                      uint32_t accumulate) {
+  if (F8 && CG == 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else if (F8)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else if (CG == 1)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
@@ -136,6 +151,12 @@ __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+// Instruction descriptor of tcgen05.mma kind::f8f6f4 with E4M3 operands: D = f32 (bits 4-5
+// = 1), A and B format E4M3 (code 0), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
 // 32 lanes x NCOL consecutive 32-bit TMEM columns -> NCOL registers per thread.
 template <int NCOL>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t* r);
@@ -163,17 +184,25 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t* r) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Output value of one accumulator: ((float)acc * sx) * sw, each product rounded.
-__device__ __forceinline__ float dequant(int32_t acc, float sxm, float swn) {
-  return __fmul_rn(__fmul_rn(__int2float_rn(acc), sxm), swn);
+// The accumulator as binary32: an int32 rounded to nearest, or (F8) the fp32 bits as they are.
+template <bool F8>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+  return F8 ? __uint_as_float(r) : __int2float_rn((int32_t)r);
 }
 
-__device__ __forceinline__ void store_out(const GemmParams& p, int64_t m, int64_t n, int32_t acc, float sxm,
+// Output value of one accumulator: ((float)acc * sx) * sw, each product rounded.
+template <bool F8>
+__device__ __forceinline__ float dequant(uint32_t acc, float sxm, float swn) {
+  return __fmul_rn(__fmul_rn(acc_value<F8>(acc), sxm), swn);
+}
+
+template <bool F8>
+__device__ __forceinline__ void store_out(const GemmParams& p, int64_t m, int64_t n, uint32_t acc, float sxm,
                                           float swn) {
   const int64_t off = m * p.ldy + n;
-  if (p.ydt == SQ_BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(dequant(acc, sxm, swn));
-  else if (p.ydt == SQ_F32) reinterpret_cast<float*>(p.y)[off] = dequant(acc, sxm, swn);
-  else reinterpret_cast<int32_t*>(p.y)[off] = acc;
+  if (p.ydt == SQ_BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(dequant<F8>(acc, sxm, swn));
+  else if (p.ydt == SQ_F32) reinterpret_cast<float*>(p.y)[off] = dequant<F8>(acc, sxm, swn);
+  else reinterpret_cast<int32_t*>(p.y)[off] = (int32_t)acc;
 }
 
 // Unit u -> (A tile, B tile, K split).  Splits of one tile are adjacent so they run
@@ -221,7 +250,7 @@ struct GemmSmem {
 // the B tile, signalling the leader's (rank 0) full barrier; the leader issues the pair MMAs
 // and its commits arrive on the barriers of both CTAs; each CTA's epilogue drains its own
 // TMEM (its 128 rows x BN columns) and arrives on the leader's accumulator-empty barrier.
-template <int BN, int STAGES, bool SWAP, int CG>
+template <int BN, int STAGES, bool SWAP, int CG, bool F8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  const GemmParams p) {
@@ -229,7 +258,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M = 128 needs N % 16 == 0, 16..256");
   static_assert(CG == 1 || (!SWAP && BN % 32 == 0), "the pair path runs the non-swapped layout, N % 32 == 0");
   constexpr int MMA_M = BM * CG;
-  constexpr uint32_t IDESC = idesc_i8(MMA_M, BN);
+  constexpr uint32_t IDESC = F8 ? idesc_e4m3(MMA_M, BN) : idesc_i8(MMA_M, BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -353,7 +382,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           const uint32_t sb = sa + L::A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
-            tc_mma_i8<CG>(d_tmem, sw128_desc(sa + k * UMMA_K), sw128_desc(sb + k * UMMA_K), IDESC,
+            tc_mma<CG, F8>(d_tmem, sw128_desc(sa + k * UMMA_K), sw128_desc(sb + k * UMMA_K), IDESC,
                           (kb > kb0 || k > 0) ? 1u : 0u);
           }
           if (CG == 1) tc_commit(empty_bar(stage));
@@ -407,8 +436,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 uint32_t packed[CH / 2];
 #pragma unroll
                 for (int i = 0; i < CH; i += 2) {
-                  const float v0 = dequant((int32_t)r[i], sxm, __ldg(p.sw + n0 + i));
-                  const float v1 = dequant((int32_t)r[i + 1], sxm, __ldg(p.sw + n0 + i + 1));
+                  const float v0 = dequant<F8>(r[i], sxm, __ldg(p.sw + n0 + i));
+                  const float v1 = dequant<F8>(r[i + 1], sxm, __ldg(p.sw + n0 + i + 1));
                   __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(v0), __float2bfloat16_rn(v1));
                   packed[i / 2] = *reinterpret_cast<uint32_t*>(&h);
                 }
@@ -419,7 +448,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
               } else {
                 for (int i = 0; i < CH; ++i) {
                   const int64_t n = n0 + i;
-                  if (n < p.N) store_out(p, m, n, (int32_t)r[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n));
+                  if (n < p.N) store_out<F8>(p, m, n, r[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n));
                 }
               }
             }
@@ -438,7 +467,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
               const float swn = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n);
               for (int i = 0; i < CH; ++i) {
                 const int64_t m = m0 + i;
-                if (m < p.M) store_out(p, m, n, (int32_t)r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
+                if (m < p.M) store_out<F8>(p, m, n, r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
               }
             }
           }
@@ -471,22 +500,32 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 }
 
 
-// Sums the split-K int32 partials in split order (exact) and applies the epilogue.
+// Sums the split-K partials in split order (int32: exact; F8: fp32 in that fixed order) and
+// applies the epilogue.
+template <bool F8>
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(const int32_t* __restrict__ ws, int splits, int64_t M, int64_t N, const float* __restrict__ sx,
                      const float* __restrict__ sw, void* __restrict__ y, int64_t ldy, int ydt) {
   const int64_t total = M * N;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    int32_t acc = 0;
-    for (int s = 0; s < splits; ++s) acc += ws[(int64_t)s * total + i];
+    uint32_t acc;
+    if (F8) {
+      float a = 0.0f;
+      for (int s = 0; s < splits; ++s) a = __fadd_rn(a, __int_as_float(ws[(int64_t)s * total + i]));
+      acc = __float_as_uint(a);
+    } else {
+      int32_t a = 0;
+      for (int s = 0; s < splits; ++s) a += ws[(int64_t)s * total + i];
+      acc = (uint32_t)a;
+    }
     const int64_t m = i / N, n = i % N;
     const int64_t off = m * ldy + n;
     if (ydt == SQ_BF16)
-      reinterpret_cast<__nv_bfloat16*>(y)[off] = __float2bfloat16_rn(dequant(acc, __ldg(sx + m), __ldg(sw + n)));
+      reinterpret_cast<__nv_bfloat16*>(y)[off] = __float2bfloat16_rn(dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n)));
     else if (ydt == SQ_F32)
-      reinterpret_cast<float*>(y)[off] = dequant(acc, __ldg(sx + m), __ldg(sw + n));
+      reinterpret_cast<float*>(y)[off] = dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n));
     else
-      reinterpret_cast<int32_t*>(y)[off] = acc;
+      reinterpret_cast<int32_t*>(y)[off] = (int32_t)acc;
   }
 }
 
@@ -540,16 +579,6 @@ struct GemmPlan {
   size_t ws_bytes;
 };
 
-// Pair tiles unless SQ_GEMM_PAIR=0 is set in the environment (read once; a tuning aid).
-static bool pairs_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("SQ_GEMM_PAIR");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
-}
-
 static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
   GemmPlan pl{};
   const int sms = num_sms();
@@ -561,7 +590,7 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
     pl.tiles_b = 1;
   } else {
     pl.bn = 256;
-    pl.cg = pairs_enabled() ? 2 : 1;
+    pl.cg = 2;
     const int64_t tile_m = (int64_t)sqk::BM * pl.cg;
     pl.tiles_a = (int)((M + tile_m - 1) / tile_m);
     pl.tiles_b = (int)((N + pl.bn - 1) / pl.bn);
@@ -582,11 +611,11 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K) { return plan_gemm(M, N, K).ws_bytes; }
 
-template <int BN, int STAGES, bool SWAP, int CG>
+template <int BN, int STAGES, bool SWAP, int CG, bool F8>
 static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const sqk::GemmParams& p,
                               cudaStream_t st) {
   using L = sqk::GemmSmem<BN, STAGES, CG>;
-  auto kern = sqk::w8a8_gemm_kernel<BN, STAGES, SWAP, CG>;
+  auto kern = sqk::w8a8_gemm_kernel<BN, STAGES, SWAP, CG, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
   if (e != cudaSuccess) return e;
   const int slots = num_sms() / CG;
@@ -610,9 +639,10 @@ static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, cons
   return cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
 }
 
-cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
-                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
-                        bool* ws_too_small) {
+template <bool F8>
+static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* wq, const float* sw, int64_t M,
+                                   int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
+                                   cudaStream_t st, bool* ws_too_small) {
   const GemmPlan pl = plan_gemm(M, N, K);
   *ws_too_small = pl.ws_bytes > 0 && (ws == nullptr || ws_bytes < pl.ws_bytes);
   if (*ws_too_small) return cudaSuccess;
@@ -658,21 +688,34 @@ cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, con
   p.ws = static_cast<int32_t*>(ws);
   cudaError_t e;
   if (!pl.swap) {
-    e = pl.cg == 2 ? launch_cfg<256, 6, false, 2>(ma, mb, p, st) : launch_cfg<256, 4, false, 1>(ma, mb, p, st);
+    e = launch_cfg<256, 6, false, 2, F8>(ma, mb, p, st);
   } else {
     switch (pl.bn) {
-      case 16: e = launch_cfg<16, 10, true, 1>(ma, mb, p, st); break;
-      case 32: e = launch_cfg<32, 9, true, 1>(ma, mb, p, st); break;
-      case 64: e = launch_cfg<64, 8, true, 1>(ma, mb, p, st); break;
-      default: e = launch_cfg<128, 6, true, 1>(ma, mb, p, st); break;
+      case 16: e = launch_cfg<16, 10, true, 1, F8>(ma, mb, p, st); break;
+      case 32: e = launch_cfg<32, 9, true, 1, F8>(ma, mb, p, st); break;
+      case 64: e = launch_cfg<64, 8, true, 1, F8>(ma, mb, p, st); break;
+      default: e = launch_cfg<128, 6, true, 1, F8>(ma, mb, p, st); break;
     }
   }
   if (e != cudaSuccess || pl.splits == 1) return e;
   const int64_t total = M * N;
   const int64_t grid = std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 16);
-  sqk::splitk_reduce_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const int32_t*>(ws), pl.splits, M, N, sx,
-                                                            sw, y, ldy, ydt);
+  sqk::splitk_reduce_kernel<F8><<<(unsigned)grid, 256, 0, st>>>(static_cast<const int32_t*>(ws), pl.splits, M, N,
+                                                                sx, sw, y, ldy, ydt);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
+                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
+                        bool* ws_too_small) {
+  return launch_gemm_any<false>(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, ws_bytes, st, ws_too_small);
+}
+
+// FP8 variant: E4M3 codes, fp32 accumulation, the same epilogue (ydt BF16 or F32).
+cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw, int64_t M,
+                            int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
+                            cudaStream_t st, bool* ws_too_small) {
+  return launch_gemm_any<true>(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, ws_bytes, st, ws_too_small);
 }
 
 // Device address of the error word on the current device (for kernels in other files).

@@ -19,7 +19,8 @@ namespace sqk {
 // loads are issued before the current row is reduced, so HBM stays busy during the
 // block-wide reductions.  With KEEP_Y the row's y values stay in registers between the
 // absmax and the quantisation (computed once); otherwise they are recomputed.
-template <bool BF16, int MAXC, bool LN, bool PREFETCH, bool KEEP_Y>
+// F8: E4M3 codes with scale = max / 448 (the FP8 variant) instead of INT8 with max / 127.
+template <bool BF16, int MAXC, bool LN, bool PREFETCH, bool KEEP_Y, bool F8 = false>
 __global__ void __launch_bounds__(ROW_THREADS)
 ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
                        const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
@@ -54,7 +55,7 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
       }
     }
     amax = block_max(amax, red + 2 * (ROW_WARPS + 1));
-    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, 127.0f);
+    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, F8 ? 448.0f : 127.0f);
     const SharedDivisor d(scale);
     if (threadIdx.x == 0) sx[m] = scale;
     int8_t* qrow = xq + m * (int64_t)K;
@@ -72,7 +73,10 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
           if (LN) ln_chunk(f, mu, rstd, gamma_f, beta_f, c, y);
           else div_chunk(f, s, c, y);
         }
-        *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false, true>(y, d);
+        if (F8)
+          *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = d.fast ? pack8_e4m3<true>(y, d) : pack8_e4m3<false>(y, d);
+        else
+          *reinterpret_cast<uint2*>(qrow + (int64_t)c * 8) = pack8_codes<false, true>(y, d);
       }
     }
     if (PREFETCH) cur = nxt;
@@ -220,13 +224,13 @@ int pick_row_threads(int64_t K, int max_nch, int* nch) {
   return 0;
 }
 
-template <bool BF16, int MAXC, bool LN>
+template <bool BF16, int MAXC, bool LN, bool F8 = false>
 static cudaError_t launch_lnq_mode(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                    const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                    const float* scale_in, int write_codes, cudaStream_t st) {
   constexpr bool PF = BF16 && MAXC <= 4;      // register double buffer while it stays small
   constexpr bool KEEP = MAXC <= 8;            // y in registers (64 floats at most)
-  auto kern = sqk::ln_smooth_quant_kernel<BF16, MAXC, LN, PF, KEEP>;
+  auto kern = sqk::ln_smooth_quant_kernel<BF16, MAXC, LN, PF, KEEP, F8>;
   int per_sm = 1;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sqk::ROW_THREADS, 0);
   if (e != cudaSuccess) return e;
@@ -236,13 +240,15 @@ static cudaError_t launch_lnq_mode(const void* x, int64_t M, int K, int64_t ld_b
   return cudaGetLastError();
 }
 
-template <bool BF16, int MAXC>
+template <bool BF16, int MAXC, bool F8 = false>
 static cudaError_t launch_lnq_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* gamma_f,
                                 const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                 const float* scale_in, int write_codes, cudaStream_t st) {
   if (gamma_f)
-    return launch_lnq_mode<BF16, MAXC, true>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st);
-  return launch_lnq_mode<BF16, MAXC, false>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st);
+    return launch_lnq_mode<BF16, MAXC, true, F8>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in,
+                                                 write_codes, st);
+  return launch_lnq_mode<BF16, MAXC, false, F8>(x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in,
+                                                write_codes, st);
 }
 
 bool rowpipe_shape(int64_t K, bool bf16, int max_nch, int* T, int* nch);
@@ -253,7 +259,7 @@ cudaError_t launch_rowpipe_quant(const void* x, bool bf16, int64_t M, int64_t K,
 bool rowpair_supported(int64_t K, bool bf16, bool calib, int64_t rows);
 cudaError_t launch_rowpair_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
-                                 const float* scale_in, int write_codes, cudaStream_t st);
+                                 const float* scale_in, int write_codes, bool f8, cudaStream_t st);
 
 // One pass of the row quantiser: per-token scales (scale_in == NULL) or a given per-tensor
 // scale; write_codes = 0 computes the per-token scales only.
@@ -262,7 +268,7 @@ static cudaError_t launch_rows(const void* x, bool bf16, int64_t M, int64_t K, i
                                const float* scale_in, int write_codes, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   if (rowpair_supported(K, bf16, false, M))  // chunk-pair rows of the model widths
-    return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, st);
+    return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, false, st);
   int pT = 0, pn = 0;
   if (K <= 8192 && rowpipe_shape(K, bf16, 4, &pT, &pn))  // staged rows, 4 chunks per thread
     return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, scale_in, write_codes,
@@ -296,6 +302,28 @@ cudaError_t launch_ln_smooth_quant(const void* x, bool bf16, int64_t M, int64_t 
                                    const float* gamma_f, const float* beta_f, const float* s, float eps,
                                    int8_t* xq, float* sx, cudaStream_t st) {
   return launch_rows(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, nullptr, 1, st);
+}
+
+// FP8 variant (per-token E4M3 codes, scale = max / 448): the chunk-pair row kernels for the
+// model widths, the block-per-row kernel otherwise.
+cudaError_t launch_ln_smooth_quant_fp8(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,
+                                       const float* gamma_f, const float* beta_f, const float* s, float eps,
+                                       uint8_t* xq, float* sx, cudaStream_t st) {
+  int8_t* q = reinterpret_cast<int8_t*>(xq);
+  if (rowpair_supported(K, bf16, false, M))
+    return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, q, sx, nullptr, 1, true, st);
+  const int64_t ldb = ldx * (bf16 ? 2 : 4);
+  const int need = (int)((K / 8 + sqk::ROW_THREADS - 1) / sqk::ROW_THREADS);
+  const int k = (int)K;
+#define SQ_LNQ8_CASE(C)                                                                                      \
+  if (need <= C)                                                                                             \
+    return bf16 ? launch_lnq_t<true, C, true>(x, M, k, ldb, gamma_f, beta_f, s, eps, q, sx, nullptr, 1, st) \
+                : launch_lnq_t<false, (C > 16 ? 16 : C), true>(x, M, k, ldb, gamma_f, beta_f, s, eps, q, sx,   \
+                                                               nullptr, 1, st);
+  SQ_LNQ8_CASE(1) SQ_LNQ8_CASE(2) SQ_LNQ8_CASE(4) SQ_LNQ8_CASE(8) SQ_LNQ8_CASE(16) SQ_LNQ8_CASE(24)
+  SQ_LNQ8_CASE(32)
+#undef SQ_LNQ8_CASE
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_ln_smooth_quant_per_tensor(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx,

@@ -132,6 +132,34 @@ __device__ __forceinline__ float pair_group_max(float m, float* red, int t, int 
   return r;
 }
 
+// E4M3 codes of the 16 values of one chunk pair (the FP8 variant): the same quotient with the
+// dividend's sign kept on zero results, then the saturating conversion; c0 gets the .x halves.
+__device__ __forceinline__ void pair_codes_e4m3(const float2* v, const SharedDivisor& d, uint2& c0, uint2& c1) {
+  float lo[8], hi[8];
+  if (d.fast) {
+    if (d.y == 0.0f) {  // zero scale: +0 codes
+      c0 = c1 = make_uint2(0u, 0u);
+      return;
+    }
+    const float2 rc = make_float2(d.y, d.y), nb = make_float2(-d.b, -d.b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 q = __fmul2_rn(v[e], rc);
+      const float2 qq = __ffma2_rn(__ffma2_rn(q, nb, v[e]), rc, q);
+      lo[e] = with_sign_of(qq.x, v[e].x);
+      hi[e] = with_sign_of(qq.y, v[e].y);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      lo[e] = d.div(v[e].x);
+      hi[e] = d.div(v[e].y);
+    }
+  }
+  c0 = make_uint2(e4m3x4(lo[0], lo[1], lo[2], lo[3]), e4m3x4(lo[4], lo[5], lo[6], lo[7]));
+  c1 = make_uint2(e4m3x4(hi[0], hi[1], hi[2], hi[3]), e4m3x4(hi[4], hi[5], hi[6], hi[7]));
+}
+
 // Codes of the 16 values of one chunk pair with a shared scale (Markstein quotient and the
 // rounding add of sq_common.cuh, on packed pairs); c0 gets the .x halves, c1 the .y halves.
 template <bool CLAMP>
@@ -169,8 +197,9 @@ __device__ __forceinline__ void pair_codes_slow(const float2* v, const SharedDiv
 
 // bf16 rows of K = 8 T NCH elements.  vec_a / vec_b: gamma' / beta' (LN_QUANT, beta' may be
 // NULL), s / unused (PLAIN_QUANT), gamma / beta (LN_CALIB).  scale_in: the per-tensor scale
-// (codes clamp), else per-token scales; write_codes = 0 writes sx only.
-template <int T, int NCH, int W, int S, int MODE>
+// (codes clamp), else per-token scales; write_codes = 0 writes sx only.  F8: E4M3 codes with
+// scale = max / 448 (the FP8 variant; per-token scales only).
+template <int T, int NCH, int W, int S, int MODE, bool F8 = false>
 __global__ void __launch_bounds__(32 * W, 1)
 rowpair_kernel(const char* __restrict__ x, int64_t M, int64_t ld_bytes, const float* __restrict__ vec_a,
                const float* __restrict__ vec_b, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
@@ -321,6 +350,10 @@ rowpair_kernel(const char* __restrict__ x, int64_t M, int64_t ld_bytes, const fl
           const float2 e23 = __ffma2_rn(q23, make_float2(ns.z, ns.w), x23);
           v[q][2 * h] = __ffma2_rn(e01, r01, q01);
           v[q][2 * h + 1] = __ffma2_rn(e23, r23, q23);
+          if (F8) {  // RN(-0 / s) = -0, which Markstein's correction turns into +0; E4M3 keeps the sign
+            v[q][2 * h] = make_float2(with_sign_of(v[q][2 * h].x, x01.x), with_sign_of(v[q][2 * h].y, x01.y));
+            v[q][2 * h + 1] = make_float2(with_sign_of(v[q][2 * h + 1].x, x23.x), with_sign_of(v[q][2 * h + 1].y, x23.y));
+          }
         }
     } else {  // a divisor outside Markstein's range somewhere in s
 #pragma unroll
@@ -351,9 +384,14 @@ rowpair_kernel(const char* __restrict__ x, int64_t M, int64_t ld_bytes, const fl
     float amax = fmax3(am[0], am[1], fmaxf(am[2], am[3]));
     amax = pair_group_max<T>(amax, red[gid] + 16, t, gid);
     if (!LN) issue(slot, r + S * rstep);  // this thread's share of the slot is in registers
-    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, 127.0f);
+    const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(amax, F8 ? 448.0f : 127.0f);
     if (t == 0) sx[r] = scale;
-    if (write_codes) {
+    if (F8) {
+      const SharedDivisor d(scale);
+      uint2* q0 = reinterpret_cast<uint2*>(xq + r * (int64_t)K) + t;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) pair_codes_e4m3(v[q], d, q0[2 * T * q], q0[2 * T * q + T]);
+    } else if (write_codes) {
       const SharedDivisor d(scale);
       const bool clamp = scale_in != nullptr;
       int8_t* qrow = xq + r * (int64_t)K;
@@ -404,14 +442,14 @@ static constexpr size_t rowpair_smem(int K, int G, int S) {
   return 128 + (size_t)K * 8 + (size_t)G * S * K * 2;
 }
 
-template <int T, int NCH, int W, int S, int MODE>
+template <int T, int NCH, int W, int S, int MODE, bool F8>
 static cudaError_t launch_rowpair(const void* x, int64_t M, int64_t ld_bytes, const float* va, const float* vb,
                                   float eps, int8_t* xq, float* sx, float* out, const float* scale_in,
                                   int write_codes, cudaStream_t st) {
   constexpr int G = 32 * W / T;
   constexpr size_t smem = rowpair_smem(8 * T * NCH, G, S);
   static_assert(smem + sizeof(float) * G * 24 <= 227 * 1024, "block exceeds the shared memory of an SM");
-  auto kern = sqk::rowpair_kernel<T, NCH, W, S, MODE>;
+  auto kern = sqk::rowpair_kernel<T, NCH, W, S, MODE, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 1;
@@ -437,13 +475,13 @@ bool rowpair_supported(int64_t K, bool bf16, bool calib, int64_t rows) {
   }
 }
 
-template <int MODE>
+template <int MODE, bool F8 = false>
 static cudaError_t launch_rowpair_mode(int64_t K, const void* x, int64_t M, int64_t ldb, const float* va,
                                        const float* vb, float eps, int8_t* xq, float* sx, float* out,
                                        const float* scale_in, int write_codes, cudaStream_t st) {
   constexpr bool CAL = MODE == sqk::PAIR_LN_CALIB;
 #define SQ_PAIR(T, NCH, W, S) \
-  launch_rowpair<T, NCH, W, S, MODE>(x, M, ldb, va, vb, eps, xq, sx, out, scale_in, write_codes, st)
+  launch_rowpair<T, NCH, W, S, MODE, F8>(x, M, ldb, va, vb, eps, xq, sx, out, scale_in, write_codes, st)
   switch (K) {
     case 512: return SQ_PAIR(32, 2, 16, 2);
     case 1024: return SQ_PAIR(64, 2, 16, 2);
@@ -465,8 +503,15 @@ static cudaError_t launch_rowpair_mode(int64_t K, const void* x, int64_t M, int6
 
 cudaError_t launch_rowpair_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
-                                 const float* scale_in, int write_codes, cudaStream_t st) {
+                                 const float* scale_in, int write_codes, bool f8, cudaStream_t st) {
   const int64_t ldb = ldx * 2;
+  if (f8) {
+    if (gamma_f)
+      return launch_rowpair_mode<sqk::PAIR_LN_QUANT, true>(K, x, M, ldb, gamma_f, beta_f, eps, xq, sx, nullptr,
+                                                           nullptr, 1, st);
+    return launch_rowpair_mode<sqk::PAIR_PLAIN_QUANT, true>(K, x, M, ldb, s, nullptr, eps, xq, sx, nullptr, nullptr,
+                                                            1, st);
+  }
   if (gamma_f)
     return launch_rowpair_mode<sqk::PAIR_LN_QUANT>(K, x, M, ldb, gamma_f, beta_f, eps, xq, sx, nullptr, scale_in,
                                                    write_codes, st);
