@@ -286,6 +286,48 @@ def fp8_gemm(xq: np.ndarray, sx: np.ndarray, wq: np.ndarray, sw: np.ndarray, out
     return acc, y
 
 
+# ----------------------------------------------------------------------------- alpha search
+def alpha_grid(n: int = 20) -> np.ndarray:
+    """n migration strengths evenly covering [0, 1] (both ends included)."""
+    return np.linspace(0.0, 1.0, n).astype(np.float32)
+
+
+def alpha_search(x: np.ndarray, W: np.ndarray, alphas, gamma=None, beta=None, eps: float = 1e-5):
+    """Migration strength by grid search on calibration data.
+
+    "4.2 W8A8 量化与 SmoothQuant" sec. 5.2: alpha is fixed once, offline, by a grid search on
+    calibration samples; "量化：只压权重，与训练后量化（PTQ）", AWQ paragraph: the search
+    objective is the layer-output error || Q(W diag(s)) (diag(s)^-1 X) - W X || over a grid
+    of alpha in [0, 1].  (The paper's own criterion, validation perplexity, needs a model and
+    data; the layer-output error is the objective the pages give for a data-only search.)
+
+    For each alpha: s = smooth_factors(ax, aw, alpha) with ax the calibration absmax of the
+    layer input (LN(x; gamma, beta) when gamma is given, else x) and aw the weight row absmax;
+    the W8A8 layer of this oracle (fold, per-token quantiser, INT8 GEMM, binary32 epilogue
+    ((float)acc * sx) * sw); err = ||Y_hat - Y||_F^2 / ||Y||_F^2 with Y = X_in W in float64.
+    Returns err [len(alphas)] (float64)."""
+    alphas = np.asarray(alphas, np.float32)
+    x, W = _c(x), _c(W)
+    if gamma is not None:
+        x_in = layernorm(x, gamma, beta, eps)
+        ax = calib_absmax(x_in, 0)
+    else:
+        x_in = bf16_to_f32(x) if x.dtype == np.uint16 else x
+        ax = calib_absmax(x, 0)
+    aw = calib_absmax(W, 1)
+    W32 = bf16_to_f32(W) if W.dtype == np.uint16 else W
+    Y = x_in.astype(np.float64) @ W32.astype(np.float64)
+    den = float(np.sum(Y * Y))
+    out = np.empty(alphas.size, np.float64)
+    for i, a in enumerate(alphas):
+        s = smooth_factors(ax, aw, float(a))
+        wq, sw, gf, bf = fold_quant_weights(W, s, gamma, beta)
+        xq, sx = ln_smooth_quant(x, gamma_f=gf, beta_f=bf, eps=eps) if gamma is not None else ln_smooth_quant(x, s=s)
+        yh = w8a8_gemm(xq, sx, wq, sw, "f32").astype(np.float64)
+        out[i] = float(np.sum((yh - Y) ** 2)) / den
+    return out
+
+
 # ----------------------------------------------------------------------------- binary64 definitions
 def smooth_transform_f64(X: np.ndarray, W: np.ndarray, s: np.ndarray):
     """X' = X diag(s)^-1 (columns divided), W' = diag(s) W (rows scaled), in float64."""

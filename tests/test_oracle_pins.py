@@ -491,3 +491,28 @@ def test_fp8_smoothquant_linear_error_is_small():
     yq = acc * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
     Y = x.astype(np.float64) @ W.astype(np.float64)
     assert _rel_fro(yq, Y) < 2.0 ** -4
+
+
+# ----------------------------------------------------------------------------- alpha search
+def test_alpha_search_objective_reproduces_the_worked_example():
+    """The objective at alpha = 0.5 on the PTQ page's 3x3 example is the square of the page's
+    per-token relative error after smoothing (0.048%)."""
+    g = json.load(open(os.path.join(GOLDEN, "p4_worked_example.json")))
+    X = np.array(g["X"], np.float32)
+    W = np.array(g["W"], np.float32)
+    err = O.alpha_search(X, W, [0.5])
+    rel = float(np.sqrt(err[0]))
+    want, tol = g["rel_err_per_token_act"][1], g["rel_err_per_token_abs"][1]
+    assert abs(rel - want) <= tol, (rel, want)
+
+
+def test_alpha_search_grid_and_extremes():
+    """20 strengths over [0, 1]; on an outlier-bearing case neither extreme is the optimum
+    (alpha = 0 leaves the activation outliers, alpha = 1 moves them all into the weights)."""
+    a = O.alpha_grid(20)
+    assert a.size == 20 and a[0] == 0.0 and a[-1] == 1.0 and np.all(np.diff(a) > 0)
+    c = sq_inputs.make_case(96, 256, 64, 21, outlier_mult=60.0)
+    err = O.alpha_search(c.x, c.W, a, gamma=c.gamma)
+    best = int(np.argmin(err))
+    assert 0 < best < a.size - 1
+    assert err[best] < 0.5 * min(err[0], err[-1])
