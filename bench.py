@@ -532,7 +532,13 @@ def run_kernel(args):
         rot[0] += 1
         sq.sq_w8a8_gemm_fp8(xq, sx8, wq, sw8, y=y, workspace=L.ws)
 
+    if args.kernel == "alpha":
+        # the whole 20-strength search on this batch (calibration statistics, reference product,
+        # 20 x (factors, fold, quantiser, GEMM, error)); the workspace is allocated once
+        alpha_ws = torch.empty(sq.lib().sq_alpha_search_workspace_size(M, K, N), dtype=torch.uint8, device=device)
+
     calls = {
+        "alpha": (lambda: sq.sq_alpha_search(L.x, L.W, None, gamma=L.gamma, workspace=alpha_ws), 0, 0.0),
         "gemm": (gemm_call, gemm_bytes, 2.0 * M * N * K),
         "gemm8": (gemm8_call, gemm_bytes, 2.0 * M * N * K),
         "fold": (rotated(lambda: sq.sq_fold_quant_weights(pick(ws), L.s, L.gamma, wq=pick(wq_out), sw=L.sw,
@@ -577,8 +583,10 @@ def run_kernel(args):
     med = t[len(t) // 2]
     peaks = load_peaks()
     out = {"kernel": args.kernel, "shape": [M, N, K], "steps": args.steps, "median_us": round(med * 1e6, 2),
-           "gbs": round(nbytes / med / 1e9, 1), "hbm_frac": round(nbytes / med / 1e9 / peaks["hbm_gbs"], 3),
            "device_error": sq.sq_device_error(clear=True)}
+    if nbytes:
+        out["gbs"] = round(nbytes / med / 1e9, 1)
+        out["hbm_frac"] = round(nbytes / med / 1e9 / peaks["hbm_gbs"], 3)
     if ops:
         out["tops"] = round(ops / med / 1e12, 1)
         out["int8_frac"] = round(ops / med / 1e12 / (INT8_PER_BF16 * peaks["bf16_tflops"]), 3)
@@ -592,7 +600,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=("gemm", "gemm8", "fold", "lnquant", "quant", "calib", "wabsmax", "xabsmax"),
+    ap.add_argument("--kernel", choices=("alpha", "gemm", "gemm8", "fold", "lnquant", "quant", "calib", "wabsmax", "xabsmax"),
                     help="run only this kernel on --shape M,N,K (profiling aid; prints no bench line)")
     ap.add_argument("--shape", default="2048,4096,4096")
     args = ap.parse_args()

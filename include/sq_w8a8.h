@@ -177,6 +177,33 @@ sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* sx, const int8_t* 
                                int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                                void* stream);
 
+/* sq_alpha_search -- migration strength by grid search on calibration data ("4.2 W8A8…"
+ * sec. 5.2: alpha is chosen once, offline, by a grid search over calibration samples;
+ * "量化…PTQ", AWQ paragraph: the data-only objective || Q(W diag(s)) (diag(s)^-1 X) - W X ||).
+ * For each alphas[i] the W8A8 layer of this library runs on the calibration batch x:
+ *   ax = absmax of the layer input (LN(x; gamma, beta) when gamma is given, else x; as
+ *   sq_calib_ln_absmax / sq_calib_absmax), aw = weight row absmax, s = sq_smooth_factors(alpha),
+ *   the fold (gamma' = gamma / s), the per-token quantiser and the GEMM with the binary32
+ *   epilogue Y_hat = ((float)acc * sx) * sw;
+ *   err[i] = ||Y_hat - Y||_F^2 / ||Y||_F^2 with Y = X_in W accumulated in binary32 (k in
+ *   increasing order) from binary32 X_in (the LayerNorm output) and W.
+ *   x: [M, K] bf16/fp32 (ldx); gamma, beta: the layer's LayerNorm (both NULL: no LayerNorm;
+ *   beta may be NULL); W: [K, N] bf16/fp32 (ldw), row j = input channel j.  Constraints as
+ *   for the steps above (K % 16 == 0, 16-byte aligned rows).
+ *   alphas: HOST array of n_alpha values in [0, 1], 1 <= n_alpha <= 256.
+ *   err: DEVICE array of n_alpha doubles (8-byte aligned), written asynchronously.
+ *   workspace: device scratch of sq_alpha_search_workspace_size(M, K, N) bytes, 256-byte
+ *   aligned, owned by the caller; calls sharing it must be ordered on one stream.
+ *   Errors: a step's own status (nothing is rolled back; err is then undefined). */
+sq_status sq_alpha_search(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                          const float* gamma, const float* beta, float eps,
+                          const void* W, sq_dtype wdt, int64_t N, int64_t ldw,
+                          const float* alphas, int n_alpha, double* err,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of sq_alpha_search for these sizes ((size_t)-1 for invalid sizes). */
+size_t sq_alpha_search_workspace_size(int64_t M, int64_t K, int64_t N);
+
 /* ------------------------------------------------------------------------------------------
  * FP8 variant.  "量化：只压权重，与训练后量化（PTQ）" (decode roofline: W8A8 in FP8 runs on tensor
  * cores with twice the BF16 peak) and "4.2 W8A8 量化与 SmoothQuant" (closing questions: FP8 as

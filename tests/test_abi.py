@@ -175,3 +175,25 @@ def test_ln_smooth_quant_per_tensor_validation():
     args = list(ok)
     args[2] = 0
     assert f(*args) == 0                             # M = 0: nothing to do
+
+
+def test_alpha_search_validation():
+    L = sq.lib()
+    f = L.sq_alpha_search
+    ws_need = L.sq_alpha_search_workspace_size(64, 256, 128)
+    assert 0 < ws_need < (1 << 40)
+    assert L.sq_alpha_search_workspace_size(64, 250, 128) == (1 << 64) - 1   # K % 16 != 0
+    a = (ctypes.c_float * 3)(0.0, 0.5, 1.0)
+    bad = (ctypes.c_float * 2)(0.5, 1.5)
+    W = ctypes.c_void_p(0x40000)
+    ws = ctypes.c_void_p(0x100000)
+    err = ctypes.c_void_p(0x50000)
+    ok = (A16, BF16, 64, 256, 256, A16b, NULL, ctypes.c_float(1e-5), W, BF16, 128, 128)
+    assert f(*ok, a, 0, err, ws, ws_need, NULL) == INVALID                  # no strengths
+    assert f(*ok, a, 257, err, ws, ws_need, NULL) == INVALID                # too many
+    assert f(*ok, bad, 2, err, ws, ws_need, NULL) == INVALID                # alpha > 1
+    assert f(*ok, a, 3, NULL, ws, ws_need, NULL) == INVALID                 # no output
+    assert f(*ok, a, 3, err, ws, ws_need - 1, NULL) == WORKSPACE            # workspace too small
+    assert f(*ok, a, 3, err, ctypes.c_void_p(0x100010), ws_need, NULL) == ALIGN
+    assert f(A16, BF16, 64, 256, 256, NULL, A16c, ctypes.c_float(1e-5), W, BF16, 128, 128,
+             a, 3, err, ws, ws_need, NULL) == INVALID                       # beta without gamma

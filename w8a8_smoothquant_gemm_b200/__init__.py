@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "sq_fold_quant_weights_fp8": [P, I, I64, I64, I64, P, P, P, P, P, P, P, P],
             "sq_ln_smooth_quant_fp8": [P, I, I64, I64, I64, P, P, P, F, P, P, P],
             "sq_w8a8_gemm_fp8": [P, P, P, P, I64, I64, I64, P, I, I64, P, SZ, P],
+            "sq_alpha_search": [P, I, I64, I64, I64, P, P, F, P, I, I64, I64, P, I, P, P, SZ, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -66,6 +67,8 @@ def lib() -> ctypes.CDLL:
             fn.restype = ctypes.c_int
         L.sq_w8a8_gemm_workspace_size.argtypes = [I64, I64, I64]
         L.sq_w8a8_gemm_workspace_size.restype = SZ
+        L.sq_alpha_search_workspace_size.argtypes = [I64, I64, I64]
+        L.sq_alpha_search_workspace_size.restype = SZ
         L.sq_status_string.argtypes = [I]
         L.sq_status_string.restype = ctypes.c_char_p
         L.sq_abi_version.argtypes = []
@@ -258,6 +261,41 @@ def sq_w8a8_gemm(xq: torch.Tensor, sx: torch.Tensor | None, wq: torch.Tensor, sw
     _check("sq_w8a8_gemm", lib().sq_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
                                               y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))
     return y
+
+
+# ----------------------------------------------------------------------------- alpha search
+def alpha_grid(n: int = 20) -> list:
+    """n migration strengths evenly covering [0, 1] (both ends included)."""
+    return [i / (n - 1) for i in range(n)] if n > 1 else [0.5]
+
+
+def sq_alpha_search(x: torch.Tensor, W: torch.Tensor, alphas=None, gamma: torch.Tensor | None = None,
+                    beta: torch.Tensor | None = None, eps: float = 1e-5, workspace: torch.Tensor | None = None,
+                    stream=None):
+    """Relative squared layer-output error of the W8A8 layer on the calibration batch x for each
+    alpha (default: 20 values over [0, 1]).  Returns (err [n] float64 on the device, alphas)."""
+    x = _mat(x, "x")
+    W = _mat(W, "W")
+    M, K = x.shape
+    N = W.shape[1]
+    if W.shape[0] != K:
+        raise ValueError("x and W disagree on K")
+    _vec(gamma, K, "gamma")
+    _vec(beta, K, "beta")
+    alphas = alpha_grid() if alphas is None else [float(a) for a in alphas]
+    arr = (ctypes.c_float * len(alphas))(*alphas)
+    err = torch.empty(len(alphas), dtype=torch.float64, device=x.device)
+    need = int(lib().sq_alpha_search_workspace_size(M, K, N))
+    if need == (1 << 64) - 1:
+        raise ValueError("unsupported sizes for the alpha search")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("sq_alpha_search",
+           lib().sq_alpha_search(_ptr(x), _dt(x), M, K, x.stride(0), _ptr(gamma), _ptr(beta), float(eps), _ptr(W),
+                                 _dt(W), N, W.stride(0), arr, len(alphas), _ptr(err), _ptr(workspace), ws_bytes,
+                                 _stream(stream)))
+    return err, alphas
 
 
 # ----------------------------------------------------------------------------- FP8 (E4M3) variant
