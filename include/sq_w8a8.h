@@ -105,6 +105,20 @@ sq_status sq_fold_quant_weights(const void* W, sq_dtype dt, int64_t K, int64_t N
                                 int8_t* Wq, float* sw, float* gamma_f, float* beta_f,
                                 void* stream);
 
+/* sq_fold_next_smoothing -- the next linear's smoothing folded offline into this linear
+ * ("量化：只压权重，与训练后量化（PTQ）", SmoothQuant section: diag(s)^-1 can be folded offline into
+ * the preceding LayerNorm or linear layer, at no runtime cost; "4.2 W8A8…" sec. 6: the input of
+ * a linear comes from a LayerNorm or from the previous GEMM).  When this linear's output is the
+ * next linear's input (with no LayerNorm between), dividing this linear's per-output-channel
+ * weight scale by the next linear's factors makes its GEMM emit the smoothed input directly:
+ *   sw_out[n] = sw[n] / s_next[n]  (binary32, correctly rounded), so that
+ *   y'[m, n] = ((float)acc[m, n] * sx[m]) * sw_out[n]  is  y[m, n] / s_next[n]  up to rounding.
+ *   The next linear then folds s_next into its own weights as usual (sq_fold_quant_weights)
+ *   and quantises y' with unit factors (sq_ln_smooth_quant, plain mode, s = 1).
+ *   sw, s_next, sw_out: fp32 [N] device arrays (sw_out may alias sw).  Works for INT8 and FP8
+ *   scales alike. */
+sq_status sq_fold_next_smoothing(const float* sw, const float* s_next, int64_t N, float* sw_out, void* stream);
+
 /* sq_ln_smooth_quant -- fused LayerNorm -> X diag(s)^-1 -> per-token INT8
  * ("4.2 W8A8…" sec. 6 and 7.1; "量化…PTQ" per-token activations):
  *   LayerNorm mode (gamma_f != NULL, s == NULL): y = LN(x) with the folded gamma' = gamma/s,

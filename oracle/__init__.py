@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.sqo_quant_per_tensor.restype = None
         L.sqo_w8a8_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I, I64]
         L.sqo_w8a8_gemm.restype = I64
+        L.sqo_fold_next_smoothing.argtypes = [P, P, I64, P]
+        L.sqo_fold_next_smoothing.restype = None
         L.sqo_e4m3_encode.argtypes = [F]
         L.sqo_e4m3_encode.restype = ctypes.c_uint8
         L.sqo_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -225,6 +227,14 @@ def w8a8_gemm(xq: np.ndarray, sx: np.ndarray, wq: np.ndarray, sw: np.ndarray, ou
     if over:
         raise OverflowError(f"{over} accumulators outside int32")
     return y
+
+
+def fold_next_smoothing(sw: np.ndarray, s_next: np.ndarray) -> np.ndarray:
+    """sw / s_next in binary32: the next linear's smoothing folded into this linear's scales."""
+    sw, s_next = _c(sw, np.float32), _c(s_next, np.float32)
+    out = np.empty_like(sw)
+    lib().sqo_fold_next_smoothing(_ptr(sw), _ptr(s_next), sw.size, _ptr(out))
+    return out
 
 
 # ----------------------------------------------------------------------------- FP8 (E4M3) variant

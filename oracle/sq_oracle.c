@@ -374,6 +374,17 @@ void sqo_quant_per_tensor(const float* y, int64_t n, int8_t* q, float* scale_out
 }
 
 /* ---------------------------------------------------------------------------
+ * The next linear's smoothing folded into this linear  [SQ-fold-prev]
+ *   "量化：只压权重，与训练后量化（PTQ）", SmoothQuant section: diag(s)^-1 folds offline into
+ *   the preceding LayerNorm or linear layer.  For a preceding linear the fold lands on its
+ *   per-output-channel scale:  sw'[n] = sw[n] / s_next[n]  (binary32), so its output
+ *   ((float)acc * sx) * sw' is the next linear's smoothed input y / s_next.
+ * ------------------------------------------------------------------------- */
+void sqo_fold_next_smoothing(const float* sw, const float* s_next, int64_t N, float* out) {
+  for (int64_t n = 0; n < N; ++n) out[n] = sw[n] / s_next[n];
+}
+
+/* ---------------------------------------------------------------------------
  * FP8 E4M3 codes  [FP8]
  *   decode: e = bits 6..3, m = bits 2..0; e = 0: (m / 8) 2^-6; else (1 + m / 8) 2^(e-7);
  *           e = 15 and m = 7: NaN

@@ -441,3 +441,41 @@ def test_per_tensor_linear_end_to_end():
     r_xq, r_sx, _ = O.ln_smooth_quant_per_tensor(c.x, gamma_f=host(gf))
     assert np.array_equal(host(xq), r_xq)
     assert assert_bf16_close(host(y), O.w8a8_gemm(r_xq, r_sx, host(wq), host(sw), "bf16")) == 1.0
+
+
+# ----------------------------------------------------------------------------- smoothing folded into the previous linear
+def test_next_smoothing_folded_into_previous_linear():
+    """Linear A feeds linear B (no LayerNorm between); B's smoothing is folded into A's output
+    scales, so A's GEMM emits B's smoothed input and B quantises it with unit factors.  Every
+    intermediate matches the oracle's chain bit for bit."""
+    rng = np.random.default_rng(12)
+    M, K1, K2, N = 300, 1024, 512, 256
+    x = (rng.standard_normal((M, K1)) * np.where(rng.random(K1) < 0.02, 40.0, 1.0)).astype(np.float32)
+    WA = rng.normal(0, 0.03, (K1, K2)).astype(np.float32)
+    WB = rng.normal(0, 0.03, (K2, N)).astype(np.float32)
+    xd, WAd, WBd = dev(x), dev(WA), dev(WB)
+    sA = sq.sq_smooth_factors(sq.sq_calib_absmax(xd, 0), sq.sq_calib_absmax(WAd, 1), 0.5)
+    wqA, swA, _, _ = sq.sq_fold_quant_weights(WAd, sA)
+    xqA, sxA = sq.sq_ln_smooth_quant(xd, s=sA)
+    yA = sq.sq_w8a8_gemm(xqA, sxA, wqA, swA, out_dtype=torch.float32)
+    sB = sq.sq_smooth_factors(sq.sq_calib_absmax(yA, 0), sq.sq_calib_absmax(WBd, 1), 0.5)
+    wqB, swB, _, _ = sq.sq_fold_quant_weights(WBd, sB)
+    swA2 = sq.sq_fold_next_smoothing(swA, sB)
+    yA2 = sq.sq_w8a8_gemm(xqA, sxA, wqA, swA2, out_dtype=torch.float32)
+    xqB, sxB = sq.sq_ln_smooth_quant(yA2, s=torch.ones(K2, dtype=torch.float32, device=DEV))
+    yB = sq.sq_w8a8_gemm(xqB, sxB, wqB, swB, out_dtype=torch.float32)
+
+    r_sA = O.smooth_factors(O.calib_absmax(x, 0), O.calib_absmax(WA, 1), 0.5)
+    r_wqA, r_swA, _, _ = O.fold_quant_weights(WA, r_sA)
+    r_xqA, r_sxA = O.ln_smooth_quant(x, s=r_sA)
+    r_yA = O.w8a8_gemm(r_xqA, r_sxA, r_wqA, r_swA, "f32")
+    r_sB = O.smooth_factors(O.calib_absmax(r_yA, 0), O.calib_absmax(WB, 1), 0.5)
+    r_wqB, r_swB, _, _ = O.fold_quant_weights(WB, r_sB)
+    r_swA2 = O.fold_next_smoothing(r_swA, r_sB)
+    r_yA2 = O.w8a8_gemm(r_xqA, r_sxA, r_wqA, r_swA2, "f32")
+    r_xqB, r_sxB = O.ln_smooth_quant(r_yA2, s=np.ones(K2, np.float32))
+    r_yB = O.w8a8_gemm(r_xqB, r_sxB, r_wqB, r_swB, "f32")
+    assert np.array_equal(host(sB), r_sB) and np.array_equal(host(swA2), r_swA2)
+    assert np.array_equal(host(yA2), r_yA2)
+    assert np.array_equal(host(xqB), r_xqB) and np.array_equal(host(sxB), r_sxB)
+    assert np.array_equal(host(yB), r_yB)

@@ -516,3 +516,50 @@ def test_alpha_search_grid_and_extremes():
     best = int(np.argmin(err))
     assert 0 < best < a.size - 1
     assert err[best] < 0.5 * min(err[0], err[-1])
+
+
+# ----------------------------------------------------------------------------- smoothing folded into the previous linear
+def _two_layer_chain(seed, folded):
+    """Linear A (K1 -> K2, plain input) feeding linear B (K2 -> N); B's smoothing either divides
+    its input at run time (plain mode, s_B) or is folded into A's output scales."""
+    rng = np.random.default_rng(seed)
+    M, K1, K2, N = 40, 128, 96, 64
+    x = (rng.standard_normal((M, K1)) * np.where(rng.random(K1) < 0.03, 30.0, 1.0)).astype(np.float32)
+    WA = rng.normal(0, 0.05, (K1, K2)).astype(np.float32)
+    WB = rng.normal(0, 0.05, (K2, N)).astype(np.float32)
+    sA = O.smooth_factors(O.calib_absmax(x, 0), O.calib_absmax(WA, 1), 0.5)
+    wqA, swA, _, _ = O.fold_quant_weights(WA, sA)
+    xqA, sxA = O.ln_smooth_quant(x, s=sA)
+    yA = O.w8a8_gemm(xqA, sxA, wqA, swA, "f32")                     # B's input, unsmoothed
+    sB = O.smooth_factors(O.calib_absmax(yA, 0), O.calib_absmax(WB, 1), 0.5)
+    wqB, swB, _, _ = O.fold_quant_weights(WB, sB)
+    if folded:
+        yA = O.w8a8_gemm(xqA, sxA, wqA, O.fold_next_smoothing(swA, sB), "f32")   # already y / sB
+        xqB, sxB = O.ln_smooth_quant(yA, s=np.ones(K2, np.float32))
+    else:
+        xqB, sxB = O.ln_smooth_quant(yA, s=sB)
+    return O.w8a8_gemm(xqB, sxB, wqB, swB, "f32"), xqB
+
+
+def test_fold_next_smoothing_divides_the_output_channel_scale():
+    rng = np.random.default_rng(8)
+    sw = np.exp(rng.uniform(-10, 0, 64)).astype(np.float32)
+    s = np.exp(rng.uniform(-2, 3, 64)).astype(np.float32)
+    out = O.fold_next_smoothing(sw, s)
+    assert np.array_equal(out, (sw / s).astype(np.float32))
+    # the dequantised output with the folded scale is y / s within two binary32 roundings
+    acc = rng.integers(-2 ** 20, 2 ** 20, (8, 64)).astype(np.float64)
+    sx = np.exp(rng.uniform(-6, 0, 8)).astype(np.float32)
+    y = ((acc.astype(np.float32) * sx[:, None]).astype(np.float32) * sw[None, :]).astype(np.float32)
+    y2 = ((acc.astype(np.float32) * sx[:, None]).astype(np.float32) * out[None, :]).astype(np.float32)
+    ref = y.astype(np.float64) / s[None, :].astype(np.float64)
+    assert np.all(np.abs(y2 - ref) <= 4 * np.spacing(np.abs(ref).astype(np.float32)))
+
+
+def test_folded_chain_matches_the_runtime_division():
+    """Folding B's smoothing into A changes only roundings: B's codes agree almost everywhere and
+    B's output stays within a fraction of its quantisation error."""
+    y_rt, q_rt = _two_layer_chain(3, folded=False)
+    y_fd, q_fd = _two_layer_chain(3, folded=True)
+    assert (q_rt == q_fd).mean() > 0.99
+    assert np.linalg.norm(y_fd - y_rt) / np.linalg.norm(y_rt) < 2e-3

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "sq_fold_quant_weights_fp8": [P, I, I64, I64, I64, P, P, P, P, P, P, P, P],
             "sq_ln_smooth_quant_fp8": [P, I, I64, I64, I64, P, P, P, F, P, P, P],
             "sq_w8a8_gemm_fp8": [P, P, P, P, I64, I64, I64, P, I, I64, P, SZ, P],
+            "sq_fold_next_smoothing": [P, P, I64, P, P],
             "sq_alpha_search": [P, I, I64, I64, I64, P, P, F, P, I, I64, I64, P, I, P, P, SZ, P],
         }
         for name, argt in sigs.items():
@@ -183,6 +184,19 @@ def sq_fold_quant_weights(W: torch.Tensor, s: torch.Tensor, gamma: torch.Tensor 
            lib().sq_fold_quant_weights(_ptr(W), _dt(W), K, N, W.stride(0), _ptr(s), _ptr(gamma), _ptr(beta),
                                        _ptr(wq), _ptr(sw), _ptr(gf), _ptr(bf), _stream(stream)))
     return wq, sw, gf, bf
+
+
+def sq_fold_next_smoothing(sw: torch.Tensor, s_next: torch.Tensor, out: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """sw / s_next: this linear's output scales with the next linear's smoothing folded in."""
+    N = sw.shape[0]
+    _vec(sw, N, "sw")
+    _vec(s_next, N, "s_next")
+    if out is None:
+        out = torch.empty_like(sw)
+    _check("sq_fold_next_smoothing", lib().sq_fold_next_smoothing(_ptr(sw), _ptr(s_next), N, _ptr(out),
+                                                                  _stream(stream)))
+    return out
 
 
 def sq_ln_smooth_quant(x: torch.Tensor, gamma_f: torch.Tensor | None = None, beta_f: torch.Tensor | None = None,

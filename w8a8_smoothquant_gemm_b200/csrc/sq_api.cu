@@ -26,6 +26,7 @@ cudaError_t launch_ln_smooth_quant_per_tensor(const void* x, bool bf16, int64_t 
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
                         int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
                         bool* ws_too_small);
+cudaError_t launch_fold_next_smoothing(const float* sw, const float* s_next, int64_t N, float* out, cudaStream_t st);
 cudaError_t launch_fold_quant_fp8(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
                                   const float* gamma, const float* beta, uint8_t* Wq, float* sw, float* gamma_f,
                                   float* beta_f, cudaStream_t st);
@@ -207,6 +208,13 @@ sq_status sq_smooth_factors(const float* ax, const float* aw, int64_t K, float a
   if (K == 0) return SQ_OK;
   if (!ax || !aw || !s || !aligned4(ax) || !aligned4(aw) || !aligned4(s)) return SQ_ERR_INVALID_ARG;
   return cuda_status(sqh::launch_smooth_factors(ax, aw, K, alpha, s, as_stream(stream)));
+}
+
+sq_status sq_fold_next_smoothing(const float* sw, const float* s_next, int64_t N, float* sw_out, void* stream) {
+  if (N < 0) return SQ_ERR_INVALID_ARG;
+  if (N == 0) return SQ_OK;
+  if (!sw || !s_next || !sw_out || !aligned4(sw) || !aligned4(s_next) || !aligned4(sw_out)) return SQ_ERR_INVALID_ARG;
+  return cuda_status(sqh::launch_fold_next_smoothing(sw, s_next, N, sw_out, as_stream(stream)));
 }
 
 sq_status sq_fold_quant_weights_fp8(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw, const float* s,

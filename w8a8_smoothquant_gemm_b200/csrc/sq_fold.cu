@@ -39,6 +39,16 @@ __global__ void smooth_factors_kernel(const float* __restrict__ ax, const float*
   s[j] = r;
 }
 
+// sw'[n] = RN(sw[n] / s_next[n]): the next linear's smoothing diag(s_next)^-1 folded into this
+// linear's per-output-channel scale ("量化：只压权重…", SmoothQuant section: diag(s)^-1 folds
+// offline into the preceding LayerNorm or linear layer), so this layer's output is already
+// the smoothed input of the next one.
+__global__ void fold_next_smoothing_kernel(const float* __restrict__ sw, const float* __restrict__ s_next, int64_t N,
+                                           float* __restrict__ out) {
+  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n < N) out[n] = __fdiv_rn(sw[n], s_next[n]);
+}
+
 // Loads 8 consecutive W elements (one 16-byte vector for bf16, two for fp32) as fp32.
 template <bool BF16>
 __device__ __forceinline__ void load8(const char* p, float f[8]) {
@@ -496,12 +506,21 @@ fold_stream_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t 
 
 }  // namespace sqk
 
+#ifndef SQ_FOLD_ONESHOT_BUDGET
+#define SQ_FOLD_ONESHOT_BUDGET (72 * 1024)  // shared memory per CTA of the one-shot cluster fold
+#endif
+
 namespace sqh {
 
 cudaError_t launch_smooth_factors(const float* ax, const float* aw, int64_t K, float alpha, float* s,
                                   cudaStream_t st) {
   const unsigned grid = (unsigned)((K + 255) / 256);
   sqk::smooth_factors_kernel<<<grid, 256, 0, st>>>(ax, aw, K, alpha, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold_next_smoothing(const float* sw, const float* s_next, int64_t N, float* out, cudaStream_t st) {
+  sqk::fold_next_smoothing_kernel<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(sw, s_next, N, out);
   return cudaGetLastError();
 }
 
@@ -631,7 +650,7 @@ static cudaError_t launch_fold_any(const void* W, bool bf16, int64_t K, int64_t 
                               const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
                               float* beta_f, cudaStream_t st) {
   int cw = 0, cl = 0, rk = 0;
-  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_cluster_shape(K, 72 * 1024, &cw, &cl, &rk)) {
+  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_cluster_shape(K, SQ_FOLD_ONESHOT_BUDGET, &cw, &cl, &rk)) {
     switch (cw) {
       case 64: return launch_fold_cluster_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
       case 32: return launch_fold_cluster_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
