@@ -5,10 +5,13 @@
 //   sw_k = max_j |W'_jk| / 127, Wq[k, j] = clamp(rne(W'_jk / sw_k))   (sec. 7.1: weights
 //   per output channel, static; "SmoothQuant大模型平滑量化技术" demo: max/127, round, clip)
 //
-// The fold kernel gives each block a strip of CW output channels (columns of W[K, N]).
-// Pass 1 streams the strip once from HBM for the column max; pass 2 re-reads it (the
-// strips resident at one time are sized to stay in L2) and writes the codes transposed
-// through shared memory into Wq[N, K] (K contiguous), the GEMM's K-major operand.
+// Wq is written transposed, [N, K] with K contiguous: the GEMM's K-major operand.  Three
+// kernels cover the shapes:
+//   fold_cluster_kernel  bf16 W whose K / 16 rows per CTA fit 72 KB of shared memory: one
+//                        pass over HBM, column maxima exchanged in a thread-block cluster;
+//   fold_l2_*            taller bf16 W (large K): chunks of output channels sized to stay
+//                        in L2, a max pass then a codes pass that re-reads the chunk from L2;
+//   fold_quant_kernel    fp32 or unaligned W: one block per strip, two passes.
 #include <algorithm>
 
 #include "sq_ptx.cuh"
@@ -388,127 +391,95 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
   fold_write_codes<CW, F8>(tile, s_rows, scale, K, N, RK, j0, k0, Wq);
 }
 
-// Fold for tall blocks (large K, where one strip's block of a CTA takes most of the shared
-// memory): clusters stay resident and walk over strips (strip = cluster, cluster +
-// clusters, ...), with two tile buffers per CTA.  Iteration i: column max of strip i,
-// partials pushed to every peer, cluster-barrier arrive | codes of strip i-1 (its scales
-// are known) | cluster-barrier wait, scales of strip i | load of strip i+1 into the buffer
-// strip i-1 used.  The cluster barrier's latency is covered by the previous strip's codes.
-template <int CW, bool F8>
+// ---------------------------------------------------------------------------- L2-blocked fold
+// Two passes over a chunk of output channels sized to stay in L2 (~40 MB of W), so W crosses
+// HBM once: pass 1 reduces max_j |s_j W_jk| of each column into sw[k] (float bits, atomicMax
+// over 256-row tiles); pass 2 re-reads the chunk (from L2), forms the scales and writes the
+// codes transposed; a last pass turns the maxima in sw into scales.  Tiles are 256 rows x 64
+// columns; no cluster or grid-wide barrier.
+template <bool BF16>
 __global__ void __launch_bounds__(256)
-fold_stream_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t N, int RK, int C,
-                    const float* __restrict__ s, const float* __restrict__ gamma, const float* __restrict__ beta,
-                    int8_t* __restrict__ Wq, float* __restrict__ sw, float* __restrict__ gamma_f,
-                    float* __restrict__ beta_f, unsigned int* err) {
-  constexpr int G = 256 / (CW / 8);  // row lanes of the max pass (8 columns per thread)
-  constexpr int NBUF = 2;
-  extern __shared__ uint8_t smem_raw[];
-  // TMA destinations want 128-byte alignment: round the dynamic base up (128 bytes of slack)
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const size_t tile_bytes = (size_t)RK * CW * 2;
-  float* s_rows = reinterpret_cast<float*>(smem + NBUF * tile_bytes);  // [RK]
-  __shared__ float red[G][CW + 1];
-  __shared__ float part[2][FOLD_MAX_CLUSTER][CW];  // partial maxima of every CTA, by strip parity
-  __shared__ float scale[2][CW];
-  __shared__ __align__(8) uint64_t bars[NBUF];
-
-  const int tid = threadIdx.x;
-  const uint32_t crank = cluster_ctarank();
-  const int64_t clusters = gridDim.x / C;
-  const int64_t strips = (N + CW - 1) / CW;
-  const int64_t j0 = (int64_t)crank * RK;
-  const int pieces = RK / 64;
-
-  for (int64_t j = (int64_t)blockIdx.x * 256 + tid; j < K; j += (int64_t)gridDim.x * 256) {
-    const float sj = s[j];
-    if (gamma && gamma_f) gamma_f[j] = __fdiv_rn(gamma[j], sj);
-    if (beta && beta_f) beta_f[j] = __fdiv_rn(beta[j], sj);
+fold_l2_max_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_bytes, const float* __restrict__ s,
+                   int64_t k_first, float* __restrict__ colmax, const float* __restrict__ gamma,
+                   const float* __restrict__ beta, float* __restrict__ gamma_f, float* __restrict__ beta_f) {
+  constexpr int ELT = BF16 ? 2 : 4;
+  __shared__ float red[32][64 + 1];
+  const int tid = threadIdx.x, cg = tid % 8, rl = tid / 8;
+  const int64_t k0 = k_first + (int64_t)blockIdx.x * 64 + cg * 8;
+  const int64_t j0 = (int64_t)blockIdx.y * 256;
+  if (gamma_f || beta_f) {  // the folded LayerNorm vectors, once (first chunk)
+    const int64_t nb = (int64_t)gridDim.x * gridDim.y, b = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+    for (int64_t j = b * 256 + tid; j < K; j += nb * 256) {
+      const float sj = s[j];
+      if (gamma && gamma_f) gamma_f[j] = __fdiv_rn(gamma[j], sj);
+      if (beta && beta_f) beta_f[j] = __fdiv_rn(beta[j], sj);
+    }
   }
-
-  if (tid == 0) {
-    for (int b = 0; b < NBUF; ++b) mbar_init(smem_u32(&bars[b]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  for (int i = tid; i < RK; i += 256) s_rows[i] = (j0 + i < K) ? __ldg(s + j0 + i) : 0.0f;
-  __syncthreads();
-
-  // one thread: the RK x CW block of strip number `n` of this cluster into its buffer (after
-  // a barrier that ended every generic read of that buffer)
-  const int64_t first = blockIdx.x / C;
-  auto issue = [&](int64_t n) {
-    const int buf = (int)(n % NBUF);
-    const uint32_t b = smem_u32(&bars[buf]);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(b, (uint32_t)tile_bytes);
-    const int64_t strip = first + n * clusters;
-    for (int p = 0; p < pieces; ++p)
-      tma_load_2d(smem_u32(smem + buf * tile_bytes + (size_t)p * 64 * CW * 2), &wmap, b, (int)(strip * CW),
-                  (int)(j0 + p * 64));
-  };
-  const int64_t count = first < strips ? (strips - first + clusters - 1) / clusters : 0;  // strips of this cluster
-  if (tid == 0 && count > 0) issue(0);
-
-  for (int64_t n = 0; n < count; ++n) {
-    const int buf = (int)(n % NBUF), par = (int)(n & 1);
-    const uint16_t* tile = reinterpret_cast<const uint16_t*>(smem + buf * tile_bytes);
-    if (!mbar_wait(smem_u32(&bars[buf]), (uint32_t)((n / NBUF) & 1))) atomicOr(err, ERR_FOLD_TMA_WAIT);
-
-    // ---- partial column max of |s_j W_jk| over this CTA's rows: thread = 8 columns x rows
-    // rl, rl + G, ...
-    {
-      const int cg = tid % (CW / 8), rl = tid / (CW / 8);
-      float m[8];
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (k0 < N) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m[e] = 0.0f;
-#pragma unroll 4
-      for (int j = rl; j < RK; j += G) {
-        const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
-        const float2 sj = make_float2(s_rows[j], s_rows[j]);
-        const float2 y0 = __fmul2_rn(sj, make_float2(bf16lo(w.x), bf16hi(w.x)));
-        const float2 y1 = __fmul2_rn(sj, make_float2(bf16lo(w.y), bf16hi(w.y)));
-        const float2 y2 = __fmul2_rn(sj, make_float2(bf16lo(w.z), bf16hi(w.z)));
-        const float2 y3 = __fmul2_rn(sj, make_float2(bf16lo(w.w), bf16hi(w.w)));
-        m[0] = fmaxf(m[0], fabsf(y0.x)); m[1] = fmaxf(m[1], fabsf(y0.y));
-        m[2] = fmaxf(m[2], fabsf(y1.x)); m[3] = fmaxf(m[3], fabsf(y1.y));
-        m[4] = fmaxf(m[4], fabsf(y2.x)); m[5] = fmaxf(m[5], fabsf(y2.y));
-        m[6] = fmaxf(m[6], fabsf(y3.x)); m[7] = fmaxf(m[7], fabsf(y3.y));
+    for (int i = 0; i < 8; ++i) {
+      const int64_t j = j0 + rl + 32 * i;
+      if (j < K) {
+        float f[8];
+        const char* p = W + j * ldw_bytes + k0 * ELT;
+        if (BF16) {
+          unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(p)), f);
+        } else {
+          const float4 a = __ldg(reinterpret_cast<const float4*>(p)), c = __ldg(reinterpret_cast<const float4*>(p) + 1);
+          f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = c.x; f[5] = c.y; f[6] = c.z; f[7] = c.w;
+        }
+        const float sj = __ldg(s + j);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(sj, f[e])));
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
     }
-    __syncthreads();
-    if (tid < CW) {
-      float m = red[0][tid];
-      for (int g = 1; g < G; ++g) m = fmaxf(m, red[g][tid]);
-      for (int r = 0; r < C; ++r) st_dsmem_f32(&part[par][crank][tid], (uint32_t)r, m);  // into every CTA
-    }
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    // the previous strip's codes while the partials of this one are in flight
-    if (n > 0)
-      fold_write_codes<CW, F8>(reinterpret_cast<const uint16_t*>(smem + ((n - 1) % NBUF) * tile_bytes), s_rows,
-                           scale[par ^ 1], K, N, RK, j0, (first + (n - 1) * clusters) * CW, Wq);
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // every partial of strip n is here
-    if (tid < CW) {
-      float m = 0.0f;
-      for (int r = 0; r < C; ++r) m = fmaxf(m, part[par][r][tid]);
-      const float sc = __fdiv_rn(m, F8 ? 448.0f : 127.0f);
-      scale[par][tid] = sc;
-      const int64_t k0 = (first + n * clusters) * CW;
-      if (crank == 0 && k0 + tid < N) sw[k0 + tid] = sc;
-    }
-    __syncthreads();  // scales visible; red and the previous strip's buffer free
-    if (tid == 0 && n + 1 < count) issue(n + 1);  // strip n-1's buffer is free now
   }
-  if (count > 0)
-    fold_write_codes<CW, F8>(reinterpret_cast<const uint16_t*>(smem + ((count - 1) % NBUF) * tile_bytes), s_rows,
-                         scale[(count - 1) & 1], K, N, RK, j0, (first + (count - 1) * clusters) * CW, Wq);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
+  __syncthreads();
+  if (tid < 64) {
+    float v = red[0][tid];
+    for (int r = 1; r < 32; ++r) v = fmaxf(v, red[r][tid]);
+    const int64_t k = k_first + (int64_t)blockIdx.x * 64 + tid;
+    if (k < N) atomic_max_nonneg(colmax + k, v);
+  }
 }
 
+// Pass 2 (bf16 weights): the 256 x 64 tile (from L2) into shared memory, scales from the
+// column maxima, codes written transposed (fold_write_codes).  F8: E4M3 codes, max / 448.
+template <bool F8>
+__global__ void __launch_bounds__(256)
+fold_l2_codes_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_bytes, const float* __restrict__ s,
+                     int64_t k_first, const float* __restrict__ colmax, int8_t* __restrict__ Wq) {
+  __shared__ __align__(16) uint16_t tile[256 * 64];  // W[j0 + r, kt + c] bf16 bits at r * 64 + c
+  __shared__ float s_rows[256];
+  __shared__ float scale[64];
+  const int tid = threadIdx.x, cg = tid % 8, rl = tid / 8;
+  const int64_t kt = k_first + (int64_t)blockIdx.x * 64;
+  const int64_t j0 = (int64_t)blockIdx.y * 256;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = rl + 32 * i;
+    const int64_t j = j0 + r, k = kt + cg * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (j < K && k < N) v = __ldg(reinterpret_cast<const uint4*>(W + j * ldw_bytes + k * 2));
+    *reinterpret_cast<uint4*>(tile + r * 64 + cg * 8) = v;
+  }
+  s_rows[tid] = (j0 + tid < K) ? __ldg(s + j0 + tid) : 0.0f;
+  if (tid < 64) scale[tid] = (kt + tid < N) ? __fdiv_rn(__ldg(colmax + kt + tid), F8 ? 448.0f : 127.0f) : 0.0f;
+  __syncthreads();
+  fold_write_codes<64, F8>(tile, s_rows, scale, K, N, 256, j0, kt, Wq);
+}
+
+// sw[k] = RN(max_k / 127) (F8: / 448) in place.
+template <bool F8>
+__global__ void fold_l2_scales_kernel(float* __restrict__ sw, int64_t N) {
+  const int64_t k = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (k < N) sw[k] = __fdiv_rn(sw[k], F8 ? 448.0f : 127.0f);
+}
 }  // namespace sqk
 
-#ifndef SQ_FOLD_ONESHOT_BUDGET
-#define SQ_FOLD_ONESHOT_BUDGET (72 * 1024)  // shared memory per CTA of the one-shot cluster fold
-#endif
 
 namespace sqh {
 
@@ -575,44 +546,6 @@ static cudaError_t launch_fold_cluster_t(const void* W, int64_t K, int64_t N, in
   return cudaLaunchKernelEx(&cfg, kern, map, K, N, RK, C, s, gamma, beta, Wq, sw, gamma_f, beta_f, error_word_ptr());
 }
 
-static size_t fold_stream_smem(int64_t rk, int cw) { return 128 + 2 * (size_t)rk * cw * 2 + (size_t)rk * 4; }
-
-template <int CW, bool F8>
-static cudaError_t launch_fold_stream_t(const void* W, int64_t K, int64_t N, int64_t ldw, int C, int RK,
-                                         const float* s, const float* gamma, const float* beta, int8_t* Wq,
-                                         float* sw, float* gamma_f, float* beta_f, cudaStream_t st) {
-  CUtensorMap map;
-  if (!make_tmap_2d(&map, true, W, N, K, ldw * 2, CW, 64, false)) return cudaErrorInvalidValue;
-  const size_t smem = fold_stream_smem(RK, CW);
-  auto kern = sqk::fold_stream_kernel<CW, F8>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  if (C > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  const int64_t strips = (N + CW - 1) / CW;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // as many clusters as are resident at once (each walks over strips), no more than strips
-  cfg.gridDim = dim3((unsigned)C);
-  int resident = 0;
-  e = cudaOccupancyMaxActiveClusters(&resident, kern, &cfg);
-  if (e != cudaSuccess) return e;
-  const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(strips, resident));
-  cfg.gridDim = dim3((unsigned)(clusters * C));
-  return cudaLaunchKernelEx(&cfg, kern, map, K, N, RK, C, s, gamma, beta, Wq, sw, gamma_f, beta_f, error_word_ptr());
-}
-
 // Cluster shape of the single-pass fold: C CTAs share a strip (at least 256 rows each, at
 // most 16), and the strip is the widest CW whose per-CTA block fits `budget` bytes of
 // shared memory.
@@ -630,19 +563,28 @@ static bool fold_cluster_shape(int64_t K, size_t budget, int* cw, int* c, int* r
   return false;
 }
 
-// Shape of the streaming fold (blocks taller than the one-shot fold's budget): the widest
-// CW whose two RK x CW buffers and factors fit 212 KB.
-static bool fold_stream_shape(int64_t K, int* cw, int* c, int* rk) {
-  const int cl = (int)std::min<int64_t>(16, std::max<int64_t>(1, (K + 255) / 256));
-  const int64_t rows = ((K + cl - 1) / cl + 63) / 64 * 64;
-  for (int w : {64, 32, 16})
-    if (fold_stream_smem(rows, w) <= 212 * 1024) {
-      *cw = w;
-      *c = cl;
-      *rk = (int)rows;
-      return true;
-    }
-  return false;
+// L2-blocked two-pass fold of bf16 weights: chunks of output channels whose W columns fit
+// ~40 MB, each a max pass then a codes pass (which reads the chunk again from L2).
+template <bool F8>
+static cudaError_t launch_fold_l2(const void* W, int64_t K, int64_t N, int64_t ldw, const float* s,
+                                  const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
+                                  float* beta_f, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(sw, 0, sizeof(float) * (size_t)N, st);
+  if (e != cudaSuccess) return e;
+  const int64_t ldb = ldw * 2;
+  int64_t chunk = (int64_t)(40ll << 20) / (K * 2) / 64 * 64;
+  chunk = std::max<int64_t>(64, std::min<int64_t>(chunk, (N + 63) / 64 * 64));
+  const unsigned rows = (unsigned)((K + 255) / 256);
+  for (int64_t k0 = 0; k0 < N; k0 += chunk) {
+    const int64_t kc = std::min<int64_t>(chunk, N - k0);
+    const dim3 grid((unsigned)((kc + 63) / 64), rows);
+    const bool first = k0 == 0;
+    sqk::fold_l2_max_kernel<true><<<grid, 256, 0, st>>>((const char*)W, K, N, ldb, s, k0, sw, gamma, beta,
+                                                         first ? gamma_f : nullptr, first ? beta_f : nullptr);
+    sqk::fold_l2_codes_kernel<F8><<<grid, 256, 0, st>>>((const char*)W, K, N, ldb, s, k0, sw, Wq);
+  }
+  sqk::fold_l2_scales_kernel<F8><<<(unsigned)((N + 255) / 256), 256, 0, st>>>(sw, N);
+  return cudaGetLastError();
 }
 
 template <bool F8>
@@ -650,20 +592,16 @@ static cudaError_t launch_fold_any(const void* W, bool bf16, int64_t K, int64_t 
                               const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
                               float* beta_f, cudaStream_t st) {
   int cw = 0, cl = 0, rk = 0;
-  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_cluster_shape(K, SQ_FOLD_ONESHOT_BUDGET, &cw, &cl, &rk)) {
+  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_cluster_shape(K, 72 * 1024, &cw, &cl, &rk)) {
     switch (cw) {
       case 64: return launch_fold_cluster_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
       case 32: return launch_fold_cluster_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
       default: return launch_fold_cluster_t<16, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
     }
   }
-  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_stream_shape(K, &cw, &cl, &rk)) {
-    switch (cw) {
-      case 64: return launch_fold_stream_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-      case 32: return launch_fold_stream_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-      default: return launch_fold_stream_t<16, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-    }
-  }
+  // blocks too tall for the one-shot fold (large K): the L2-blocked two-pass fold
+  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && (ldw * 2) % 16 == 0)
+    return launch_fold_l2<F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
   // narrower strips when there are few output channels, so every SM gets work
   const int64_t sms = num_sms();
   const int strip = (N / 32 >= 2 * sms) ? 32 : 16;
