@@ -96,7 +96,8 @@ def _acc_bound(xq, wq):
 
 
 GEMM_SHAPES = [(1, 8, 16), (1, 200, 272), (7, 24, 32), (16, 256, 256), (16, 4096, 4096), (64, 130, 1024),
-               (100, 1000, 512), (129, 264, 128), (256, 512, 4096), (300, 1024, 1040), (2048, 512, 96)]
+               (100, 1000, 512), (129, 264, 128), (256, 512, 4096), (300, 1024, 1040), (2048, 512, 96),
+               (5, 1000, 8192), (7, 5120, 2048)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)

@@ -288,6 +288,7 @@ GEMM_SHAPES = [
     (1, 8, 16), (1, 200, 272), (7, 24, 32), (16, 256, 256), (33, 4096, 4096), (64, 130, 1024),
     (100, 1000, 512), (128, 512, 128), (129, 264, 128), (200, 777, 400), (256, 512, 4096),
     (300, 1024, 1040), (1000, 300, 160), (2048, 512, 96),
+    (5, 1000, 8192), (7, 5120, 2048),  # decode shapes split 16 and 3 ways
 ]
 
 
