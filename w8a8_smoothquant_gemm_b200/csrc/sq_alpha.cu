@@ -54,48 +54,93 @@ __device__ __forceinline__ float load_elt(const void* p, int64_t i) {
 }
 
 // Reference product Y[M, N] = A[M, K] W[K, N] in binary32, k in increasing order per output
-// (fused multiply-add, one rounding per step).  64 x 64 output tiles, 16-deep k slabs staged
-// in shared memory, 4 x 4 outputs per thread.
+// (fused multiply-add, one rounding per step).  128 x 128 output tiles, 8-deep k slabs in
+// double-buffered shared memory, 8 x 8 outputs per thread as packed binary32 pairs (each
+// half rounds as the scalar fma would).
 template <bool ABF16, bool WBF16>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 reference_gemm_kernel(const void* __restrict__ A, int64_t lda, const void* __restrict__ W, int64_t ldw, int64_t M,
                       int64_t N, int64_t K, float* __restrict__ Y) {
-  __shared__ float As[16][64 + 4];
-  __shared__ float Ws[16][64 + 4];
+  __shared__ __align__(16) float As[2][8][128];  // [k][m]
+  __shared__ __align__(16) float Ws[2][8][128];  // [k][n]
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const int64_t m0 = (int64_t)blockIdx.y * 64, n0 = (int64_t)blockIdx.x * 64;
-  float acc[4][4] = {};
-  for (int64_t k0 = 0; k0 < K; k0 += 16) {
-    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
-      const int r = i / 16, kk = i % 16;  // A tile: 64 rows x 16 k
-      const int64_t m = m0 + r, k = k0 + kk;
-      As[kk][r] = (m < M && k < K) ? load_elt<ABF16>(A, m * lda + k) : 0.0f;
-      const int kr = i / 64, c = i % 64;  // W tile: 16 k x 64 columns
-      const int64_t k2 = k0 + kr, n = n0 + c;
-      Ws[kr][c] = (k2 < K && n < N) ? load_elt<WBF16>(W, k2 * ldw + n) : 0.0f;
+  const int64_t m0 = (int64_t)blockIdx.y * 128, n0 = (int64_t)blockIdx.x * 128;
+  // staging assignment: A tile 128 rows x 8 k (thread: row ar, k ak..ak+3), W tile 8 k x 128
+  // columns (thread: k wk, columns wc..wc+3)
+  const int ar = threadIdx.x / 2, ak = (threadIdx.x % 2) * 4;
+  const int wk = threadIdx.x / 32, wc = (threadIdx.x % 32) * 4;
+  float ra[4], rw[4];
+  // K % 8 == 0, and rows start on 16-byte boundaries: 4 consecutive elements load as one
+  // 8-byte (bf16) or 16-byte (fp32) vector
+  auto load4 = [](const void* base, int64_t i, bool bf16, float* out) {
+    if (bf16) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + i));
+      out[0] = bf16lo(u.x); out[1] = bf16hi(u.x); out[2] = bf16lo(u.y); out[3] = bf16hi(u.y);
+    } else {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i));
+      out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
     }
-    __syncthreads();
+  };
+  auto fetch = [&](int64_t k0) {
+    const int64_t m = m0 + ar;
+    if (m < M) load4(A, m * lda + k0 + ak, ABF16, ra);
+    else ra[0] = ra[1] = ra[2] = ra[3] = 0.0f;
+    const int64_t k2 = k0 + wk, n = n0 + wc;
+    if (n + 3 < N) {
+      load4(W, k2 * ldw + n, WBF16, rw);
+    } else {
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) w[j] = Ws[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(a[i], w[j], acc[i][j]);
+      for (int i = 0; i < 4; ++i) rw[i] = (n + i < N) ? load_elt<WBF16>(W, k2 * ldw + n + i) : 0.0f;
     }
-    __syncthreads();
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) As[buf][ak + i][ar] = ra[i];
+    *reinterpret_cast<float4*>(&Ws[buf][wk][wc]) = make_float4(rw[0], rw[1], rw[2], rw[3]);
+  };
+  float2 acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
+  for (int64_t k0 = 0; k0 < K; k0 += 8) {
+    const bool more = k0 + 8 < K;
+    if (more) fetch(k0 + 8);  // next slab into registers while this one is used
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
+      const float4 w0 = *reinterpret_cast<const float4*>(&Ws[buf][kk][tx * 8]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&Ws[buf][kk][tx * 8 + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float2 w[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                           make_float2(w1.z, w1.w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(make_float2(a[i], a[i]), w[j], acc[i][j]);
+    }
+    if (more) {
+      stash(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i) {
+    const int64_t m = m0 + ty * 8 + i;
+    if (m >= M) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int64_t m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
-      if (m < M && n < N) Y[m * N + n] = acc[i][j];
+      const int64_t n = n0 + tx * 8 + 2 * j;
+      if (n < N) Y[m * N + n] = acc[i][j].x;
+      if (n + 1 < N) Y[m * N + n + 1] = acc[i][j].y;
     }
+  }
 }
 
 // acc[0] += sum (Yh - Y)^2, or (Yh == NULL) sum Y^2, in binary64.
@@ -189,7 +234,7 @@ cudaError_t launch_layernorm_rows(const void* x, int64_t M, int64_t K, int64_t l
 
 cudaError_t launch_reference_gemm(const void* A, bool abf16, int64_t lda, const void* W, bool wbf16, int64_t ldw,
                                   int64_t M, int64_t N, int64_t K, float* Y, cudaStream_t st) {
-  const dim3 grid((unsigned)((N + 63) / 64), (unsigned)((M + 63) / 64));
+  const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + 127) / 128));
   if (abf16 && wbf16) sqk::reference_gemm_kernel<true, true><<<grid, 256, 0, st>>>(A, lda, W, ldw, M, N, K, Y);
   else if (abf16) sqk::reference_gemm_kernel<true, false><<<grid, 256, 0, st>>>(A, lda, W, ldw, M, N, K, Y);
   else if (wbf16) sqk::reference_gemm_kernel<false, true><<<grid, 256, 0, st>>>(A, lda, W, ldw, M, N, K, Y);

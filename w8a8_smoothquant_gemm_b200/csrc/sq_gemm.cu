@@ -445,6 +445,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
                 for (int v = 0; v < CH / 8; ++v)
                   dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+              } else if (full && p.ydt == SQ_F32) {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + m * p.ldy + n0);
+#pragma unroll
+                for (int v = 0; v < CH / 4; ++v) {  // (sw is only 4-byte aligned: scalar loads)
+                  const float* w = p.sw + n0 + 4 * v;
+                  dst[v] = make_float4(dequant<F8>(r[4 * v], sxm, __ldg(w)), dequant<F8>(r[4 * v + 1], sxm, __ldg(w + 1)),
+                                       dequant<F8>(r[4 * v + 2], sxm, __ldg(w + 2)),
+                                       dequant<F8>(r[4 * v + 3], sxm, __ldg(w + 3)));
+                }
               } else {
                 for (int i = 0; i < CH; ++i) {
                   const int64_t n = n0 + i;
