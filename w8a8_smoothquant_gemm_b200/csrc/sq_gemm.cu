@@ -269,6 +269,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::BAR_OFFSET + L::NUM_BARS * 8);
 
+  // a split-K reduction launched behind this grid may be scheduled now (it waits for this
+  // grid's completion before reading anything); without one this is a no-op
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
@@ -515,6 +518,9 @@ template <bool F8>
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(const int32_t* __restrict__ ws, int splits, int64_t M, int64_t N, const float* __restrict__ sx,
                      const float* __restrict__ sw, void* __restrict__ y, int64_t ldy, int ydt) {
+  // launched as a programmatic dependent of the GEMM: its blocks may be resident before the
+  // GEMM ends, and wait here until the GEMM grid has completed and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t total = M * N;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     uint32_t acc;
@@ -709,9 +715,18 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   if (e != cudaSuccess || pl.splits == 1) return e;
   const int64_t total = M * N;
   const int64_t grid = std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 16);
-  sqk::splitk_reduce_kernel<F8><<<(unsigned)grid, 256, 0, st>>>(static_cast<const int32_t*>(ws), pl.splits, M, N,
-                                                                sx, sw, y, ldy, ydt);
-  return cudaGetLastError();
+  // programmatic dependent launch: the reduction's launch overlaps the GEMM's tail
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sqk::splitk_reduce_kernel<F8>, static_cast<const int32_t*>(ws), pl.splits, M, N,
+                            sx, sw, y, ldy, ydt);
 }
 
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
