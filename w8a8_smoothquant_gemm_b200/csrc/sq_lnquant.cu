@@ -155,6 +155,94 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
   }
 }
 
+
+// ---------------------------------------------------------------------------- long plain rows
+// Plain mode (y = x / s) on rows too long to hold in a thread group's registers (K > 16384):
+// each row is split into 8192-element segments, one block per (row, segment).  Pass 1 folds
+// the segment's max |y| into the row's slot of sx (float bits, atomicMax; sx starts at 0);
+// pass 2 recomputes y and writes the codes with scale = RN(max / 127) (or the given
+// per-tensor scale, codes clamped); pass 3 turns the maxima in sx into scales.  y = RN(x / s)
+// is the correctly rounded division.  (Blocks that own a segment for many rows, with s and
+// RN(1/s) staged once in shared memory, measured 2.3x slower: too few loads in flight.)
+constexpr int SEG_CHUNKS = 1024;  // 8192 elements per block: 256 threads x 4 chunks of 8
+
+template <bool BF16>
+__device__ __forceinline__ void seg_load8(const char* row, int64_t c, float f[8]) {
+  if (BF16) {
+    unpack8_bf16(ldg_stream16(row + c * 16), f);
+  } else {
+    const uint4 a = ldg_stream16(row + c * 32), b = ldg_stream16(row + c * 32 + 16);
+    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y); f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+    f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y); f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256)
+rowsplit_max_kernel(const char* __restrict__ x, int64_t K, int64_t ld_bytes, int64_t nseg,
+                    const float* __restrict__ s, float* __restrict__ rowmax) {
+  __shared__ float red[8];
+  const int64_t m = (int64_t)blockIdx.x / nseg, seg = (int64_t)blockIdx.x % nseg;
+  const int64_t nchunks = K / 8;
+  const char* row = x + m * ld_bytes;
+  float am = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t c = seg * SEG_CHUNKS + i * 256 + threadIdx.x;
+    if (c < nchunks) {
+      float f[8], y[8];
+      seg_load8<BF16>(row, c, f);
+      div_chunk(f, s, (int)c, y);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(y[e]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = red[0];
+    for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w]);
+    atomic_max_nonneg(rowmax + m, v);
+  }
+}
+
+template <bool BF16, bool F8>
+__global__ void __launch_bounds__(256)
+rowsplit_codes_kernel(const char* __restrict__ x, int64_t K, int64_t ld_bytes, int64_t nseg,
+                      const float* __restrict__ s, const float* __restrict__ rowmax,
+                      const float* __restrict__ scale_in, int8_t* __restrict__ xq) {
+  const int64_t m = (int64_t)blockIdx.x / nseg, seg = (int64_t)blockIdx.x % nseg;
+  const int64_t nchunks = K / 8;
+  const char* row = x + m * ld_bytes;
+  const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(__ldg(rowmax + m), F8 ? 448.0f : 127.0f);
+  const SharedDivisor d(scale);
+  const bool clamp = scale_in != nullptr;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t c = seg * SEG_CHUNKS + i * 256 + threadIdx.x;
+    if (c < nchunks) {
+      float f[8], y[8];
+      seg_load8<BF16>(row, c, f);
+      div_chunk(f, s, (int)c, y);
+      uint2 w;
+      if (F8) w = d.fast ? pack8_e4m3<true>(y, d) : pack8_e4m3<false>(y, d);
+      else if (d.fast && !clamp) w = pack8_codes<true>(y, d);
+      else if (d.fast) w = pack8_codes<true, true>(y, d);
+      else w = pack8_codes<false, true>(y, d);
+      *reinterpret_cast<uint2*>(xq + m * K + c * 8) = w;
+    }
+  }
+}
+
+// sx[m] = RN(max_m / 127) (F8: / 448), or the given per-tensor scale.
+template <bool F8>
+__global__ void rowsplit_scales_kernel(float* __restrict__ sx, int64_t M, const float* __restrict__ scale_in) {
+  const int64_t m = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (m < M) sx[m] = scale_in ? __ldg(scale_in) : __fdiv_rn(sx[m], F8 ? 448.0f : 127.0f);
+}
+
 // out[0] = max of v[0 .. n) (non-negative floats), one block.
 __global__ void __launch_bounds__(1024) max_of_vector_kernel(const float* __restrict__ v, int64_t n, float* out) {
   __shared__ float red[32];
@@ -261,6 +349,39 @@ cudaError_t launch_rowpair_quant(const void* x, int64_t M, int64_t K, int64_t ld
                                  const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                  const float* scale_in, int write_codes, bool f8, cudaStream_t st);
 
+
+// Plain-mode rows longer than the register-resident kernels hold (see rowsplit_*).  F8: E4M3
+// codes, scale = max / 448.
+template <bool F8>
+static cudaError_t launch_rowsplit(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* s,
+                                   int8_t* xq, float* sx, const float* scale_in, int write_codes, cudaStream_t st) {
+  const int64_t ldb = ldx * (bf16 ? 2 : 4);
+  const int64_t nseg = (K / 8 + sqk::SEG_CHUNKS - 1) / sqk::SEG_CHUNKS;
+  const int64_t blocks = M * nseg;
+  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (!scale_in) {  // per-token maxima into sx
+    e = cudaMemsetAsync(sx, 0, sizeof(float) * (size_t)M, st);
+    if (e != cudaSuccess) return e;
+    if (bf16) sqk::rowsplit_max_kernel<true><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx);
+    else sqk::rowsplit_max_kernel<false><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (write_codes) {
+    if (bf16)
+      sqk::rowsplit_codes_kernel<true, F8><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx,
+                                                                            scale_in, xq);
+    else
+      sqk::rowsplit_codes_kernel<false, F8><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx,
+                                                                             scale_in, xq);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  sqk::rowsplit_scales_kernel<F8><<<(unsigned)((M + 255) / 256), 256, 0, st>>>(sx, M, scale_in);
+  return cudaGetLastError();
+}
+
 // One pass of the row quantiser: per-token scales (scale_in == NULL) or a given per-tensor
 // scale; write_codes = 0 computes the per-token scales only.
 static cudaError_t launch_rows(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,
@@ -269,6 +390,8 @@ static cudaError_t launch_rows(const void* x, bool bf16, int64_t M, int64_t K, i
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   if (rowpair_supported(K, bf16, false, M))  // chunk-pair rows of the model widths
     return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, false, st);
+  if (!gamma_f && K > 16384)  // long plain rows: split into segments, two passes
+    return launch_rowsplit<false>(x, bf16, M, K, ldx, s, xq, sx, scale_in, write_codes, st);
   int pT = 0, pn = 0;
   if (K <= 8192 && rowpipe_shape(K, bf16, 4, &pT, &pn))  // staged rows, 4 chunks per thread
     return launch_rowpipe_quant(x, bf16, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, pT, pn, scale_in, write_codes,
@@ -312,6 +435,7 @@ cudaError_t launch_ln_smooth_quant_fp8(const void* x, bool bf16, int64_t M, int6
   int8_t* q = reinterpret_cast<int8_t*>(xq);
   if (rowpair_supported(K, bf16, false, M))
     return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, q, sx, nullptr, 1, true, st);
+  if (!gamma_f && K > 16384) return launch_rowsplit<true>(x, bf16, M, K, ldx, s, q, sx, nullptr, 1, st);
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   const int need = (int)((K / 8 + sqk::ROW_THREADS - 1) / sqk::ROW_THREADS);
   const int k = (int)K;
