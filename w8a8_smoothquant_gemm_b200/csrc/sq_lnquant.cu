@@ -92,14 +92,16 @@ __global__ void __launch_bounds__(256, 2)
 ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes,
                       const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
                       const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
-                      const float* __restrict__ scale_in, int write_codes) {
+                      const float* __restrict__ scale_in, int write_codes, int use_table) {
   constexpr int G = 256 / T;
   __shared__ float red[G][24];  // per group: mean partials, variance partials, max
   extern __shared__ float rs[];  // plain mode: RN(1 / s_j), or 0 where s_j is outside the fast range
   const int gid = threadIdx.x / T, t = threadIdx.x % T;
   const int nchunks = K / 8;
-  bool all_fast = true;
-  if (!LN) {
+  // plain mode: a table of RN(1/s_j) pays off over several rows per block; with a row or two
+  // (decode) the correctly rounded division per element is cheaper than building it
+  bool all_fast = LN || use_table;
+  if (!LN && use_table) {
     int slow = 0;
     for (int j = threadIdx.x; j < K; j += 256) {
       const float a = s[j];
@@ -269,17 +271,18 @@ static cudaError_t launch_group_t(const void* x, int64_t M, int K, int64_t ld_by
                                   const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                   const float* scale_in, int write_codes, cudaStream_t st) {
   auto kern = sqk::ln_quant_group_kernel<BF16, T, NCH, LN>;
-  const size_t smem = LN ? 0 : sizeof(float) * (size_t)K;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t table = LN ? 0 : sizeof(float) * (size_t)K;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)table);
   if (e != cudaSuccess) return e;
   int per_sm = 1;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, table);
   if (e != cudaSuccess) return e;
   constexpr int G = 256 / T;
   const int64_t blocks = (M + G - 1) / G;
   const int64_t grid = std::min<int64_t>(blocks, (int64_t)num_sms() * std::max(per_sm, 1));
-  kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps, xq, sx, scale_in,
-                                          write_codes);
+  const int use_table = !LN && M >= 4 * grid * G;  // at least 4 rows per group
+  kern<<<(unsigned)grid, 256, use_table ? table : 0, st>>>((const char*)x, M, K, ld_bytes, gamma_f, beta_f, s, eps,
+                                                           xq, sx, scale_in, write_codes, use_table);
   return cudaGetLastError();
 }
 
