@@ -21,7 +21,7 @@ namespace sqk {
 
 enum RowMode : int { ROW_LN_QUANT = 0, ROW_PLAIN_QUANT = 1, ROW_LN_CALIB = 2 };
 
-template <bool BF16, int T, int NCH, int S, int MODE, bool POLL1 = false>
+template <bool BF16, int T, int NCH, int S, int MODE>
 __global__ void __launch_bounds__(256)
 rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, const float* __restrict__ vec_a,
                const float* __restrict__ vec_b, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
@@ -85,14 +85,10 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
   int64_t it = 0;
   for (int64_t r = r0; r < M; r += rstep, ++it) {
     const int slot = (int)(it % S);
-    if (POLL1) {
-      // one lane polls the slot's barrier; the rest of the group sleeps in the group barrier
-      if (t == 0 && !mbar_wait(smem_u32(&bars[gid * S + slot]), (uint32_t)((it / S) & 1)))
-        atomicOr(err, ERR_ROW_TMA_WAIT);
-      group_barrier<T>(gid);
-    } else if (!mbar_wait(smem_u32(&bars[gid * S + slot]), (uint32_t)((it / S) & 1))) {
+    // one lane polls the slot's barrier; the rest of the group sleeps in the group barrier
+    if (t == 0 && !mbar_wait(smem_u32(&bars[gid * S + slot]), (uint32_t)((it / S) & 1)))
       atomicOr(err, ERR_ROW_TMA_WAIT);
-    }
+    group_barrier<T>(gid);
     const uint8_t* rowp = gring + (size_t)slot * row_bytes;
     float v[NCH * 8];
 #pragma unroll
@@ -221,12 +217,12 @@ static size_t rowpipe_smem(int K, int elt, int G, int S) {
   return 128 + (size_t)K * 8 + (size_t)G * S * K * elt + (size_t)G * S * 8;
 }
 
-template <bool BF16, int T, int NCH, int MODE, int S, bool POLL1>
+template <bool BF16, int T, int NCH, int MODE, int S>
 static cudaError_t launch_rowpipe_v(const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
                                     const float* vb, float eps, int8_t* xq, float* sx, float* out, const float* scale_in,
                                     int write_codes, cudaStream_t st) {
   constexpr int G = 256 / T;
-  auto kern = sqk::rowpipe_kernel<BF16, T, NCH, S, MODE, POLL1>;
+  auto kern = sqk::rowpipe_kernel<BF16, T, NCH, S, MODE>;
   const size_t smem = rowpipe_smem(K, BF16 ? 2 : 4, G, S);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -246,8 +242,8 @@ template <bool BF16, int T, int NCH, int MODE>
 static cudaError_t launch_rowpipe_t(const void* x, int64_t M, int K, int64_t ld_bytes, const float* va,
                                     const float* vb, float eps, int8_t* xq, float* sx, float* out,
                                     const float* scale_in, int write_codes, cudaStream_t st) {
-  return launch_rowpipe_v<BF16, T, NCH, MODE, 2, true>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in,
-                                                       write_codes, st);
+  return launch_rowpipe_v<BF16, T, NCH, MODE, 2>(x, M, K, ld_bytes, va, vb, eps, xq, sx, out, scale_in,
+                                                 write_codes, st);
 }
 
 template <bool BF16, int T, int MODE>
