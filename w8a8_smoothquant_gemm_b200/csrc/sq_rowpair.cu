@@ -7,7 +7,7 @@
 // ("4.2 W8A8 量化与 SmoothQuant", sec. 6 and 7.1; "量化：只压权重，与训练后量化（PTQ）",
 // per-token activation quantisation), with the results of sq_rowpipe.cu bit for bit.
 //
-// Layout.  A row is handled by a group of T threads (one warp for K <= 4096).  Thread t
+// Layout.  A row is handled by a group of T threads (one to eight warps).  Thread t
 // owns the chunk pairs (c0, c1) = (2 T q + t, 2 T q + T + t), q < NCH / 2, and keeps
 // element e of both chunks in one float2, so that every per-element step (the LayerNorm
 // sums, its apply, the Markstein quotient, the rounding add) runs on packed binary32 pairs.
@@ -518,7 +518,9 @@ static cudaError_t launch_rowpair_mode(int64_t K, const void* x, int64_t M, int6
     default: break;
   }
   if constexpr (CAL) {
-    if (K == 4096) return SQ_PAIR(64, 8, 8, 2);
+    // K = 4096: four-warp groups (124 registers, 16 warps per SM) beat two-warp groups with
+    // twice the chunks (250 registers, 8 warps per SM): measured 135 against 143 us at 65536 rows
+    if (K == 4096) return SQ_PAIR(128, 4, 16, 2);
     if (K == 8192) return SQ_PAIR(128, 8, 8, 2);
   } else {
     if (K == 4096) return SQ_PAIR(64, 8, 16, 2);
