@@ -524,7 +524,12 @@ static cudaError_t launch_rowpair_mode(int64_t K, const void* x, int64_t M, int6
     if (K == 8192) return SQ_PAIR(128, 8, 8, 2);
   } else {
     if (K == 4096) return SQ_PAIR(64, 8, 16, 2);
-    if (K == 8192) return SQ_PAIR(64, 16, 8, 2);
+    if (K == 8192) {
+      // plain rows: four-warp groups with one ring slot (126 registers, 16 warps per SM)
+      // beat two-warp groups (255 registers, 8 warps per SM): 51 against 55 us at 8192 rows
+      if constexpr (MODE == sqk::PAIR_PLAIN_QUANT) return SQ_PAIR(128, 8, 16, 1);
+      return SQ_PAIR(64, 16, 8, 2);
+    }
     if (K == 12288) return SQ_PAIR(128, 12, 8, 2);
     if (K == 14336) {
       // plain rows (no reduction order): below ~4k rows, 256-thread groups (an odd 7 chunks
