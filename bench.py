@@ -185,9 +185,10 @@ class Linear:
         self.y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
         need = sq.sq_w8a8_gemm_workspace_size(M, N, K)
         self.ws = torch.empty(need, dtype=torch.uint8, device=device) if need else None
-        # this module's kernels per pass: calibration, weight absmax, factors, fold, quantiser, GEMM
-        # (+ the split-K reduction when the GEMM splits K)
-        self.launches = 6 + (1 if need else 0)
+        # this module's kernels per pass: calibration, weight absmax, factors, fold (one, or
+        # three on the streaming route), quantiser, GEMM (+ the split-K reduction when the
+        # GEMM splits K)
+        self.launches = 5 + sq.sq_fold_kernel_launches(self.W) + (1 if need else 0)
 
     def run(self, sq, world: int, ev=None):
         if self.ln:

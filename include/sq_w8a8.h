@@ -99,11 +99,20 @@ sq_status sq_smooth_factors(const float* ax, const float* aw, int64_t K, float a
  *   each written only when both its input and output pointers are non-NULL.
  *   W: [K, N] bf16/fp32 (row j = input channel), leading dimension ldw.
  *   Wq: int8 [N, K], K contiguous (the GEMM's K-major B operand), 16-byte aligned.
- *   sw: fp32 [N].  K % 16 == 0, K <= SQ_MAX_K. */
+ *   sw: fp32 [N]; it also holds the column maxima while the call runs, so it must not
+ *   alias an input.  K % 16 == 0, K <= SQ_MAX_K. */
 sq_status sq_fold_quant_weights(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw,
                                 const float* s, const float* gamma, const float* beta,
                                 int8_t* Wq, float* sw, float* gamma_f, float* beta_f,
                                 void* stream);
+
+/* sq_fold_kernel_launches -- how many kernels sq_fold_quant_weights (and
+ *   sq_fold_quant_weights_fp8) launches for these arguments: 1 for the one-pass routes,
+ *   3 for the streaming two-pass route (column maxima, codes, scales), 0 when K or N is 0.
+ *   Host only: no CUDA call, no validation beyond that (the fold itself validates).
+ *   The pages have no counterpart; it reports this library's routing, for launch
+ *   accounting by callers that count kernels. */
+int sq_fold_kernel_launches(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw);
 
 /* sq_fold_next_smoothing -- the next linear's smoothing folded offline into this linear
  * ("量化：只压权重，与训练后量化（PTQ）", SmoothQuant section: diag(s)^-1 can be folded offline into

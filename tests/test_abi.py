@@ -42,7 +42,7 @@ def test_status_strings_and_version():
     L = sq.lib()
     assert L.sq_status_string(0) == b"SQ_OK"
     assert L.sq_status_string(5) == b"SQ_ERR_WORKSPACE"
-    assert L.sq_abi_version() == 101
+    assert L.sq_abi_version() == 102
 
 
 # fake, never dereferenced device addresses with chosen alignment
@@ -197,3 +197,13 @@ def test_alpha_search_validation():
     assert f(*ok, a, 3, err, ctypes.c_void_p(0x100010), ws_need, NULL) == ALIGN
     assert f(A16, BF16, 64, 256, 256, NULL, A16c, ctypes.c_float(1e-5), W, BF16, 128, 128,
              a, 3, err, ws, ws_need, NULL) == INVALID                       # beta without gamma
+
+
+def test_fold_kernel_launches_routing():
+    f = sq.lib().sq_fold_kernel_launches
+    assert f(A16, BF16, 0, 64, 64) == 0
+    assert f(A16, BF16, 4096, 4096, 4096) == 1             # one-pass cluster fold
+    assert f(A16, BF16, 4096, 28672, 28672) == 3           # streaming two-pass fold
+    assert f(A16, BF16, 49152, 64, 64) == 3                # cluster block too tall
+    assert f(A8, BF16, 49152, 64, 64) == 1                 # unaligned: strip kernel
+    assert f(A16, F32, 4096, 28672, 28672) == 1            # fp32 weights: strip kernel

@@ -41,7 +41,8 @@ def _no_device_error():
 
 # ----------------------------------------------------------------------------- fold
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
-@pytest.mark.parametrize("K,N", [(16, 8), (256, 200), (4096, 4096), (1040, 3000), (14336, 512), (49152, 64)])
+@pytest.mark.parametrize("K,N", [(16, 8), (256, 200), (4096, 4096), (1040, 3000), (14336, 512), (49152, 64),
+                                 (40016, 1288)])
 def test_fold_fp8(dt, K, N):
     if dt == "f32" and K > 4096:
         pytest.skip("fp32 weights are covered by the smaller shapes")

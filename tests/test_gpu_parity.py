@@ -149,6 +149,23 @@ def test_fold_quant_weights(dt, K, N, extra):
     assert np.array_equal(host(gf), r[2]) and np.array_equal(host(bf), r[3])
 
 
+@pytest.mark.parametrize("K,N,extra", [(40000, 1288, 8), (49168, 1096, 0)])
+def test_fold_streaming_ragged(K, N, extra):
+    """The streaming two-pass route on a ragged last row tile and column strip, with a padded
+    leading dimension and an all-zero output channel."""
+    _, W, g, _ = sq_inputs.torch_case(1, K, N, 11, DEV, w_std=0.015)
+    W = torch.nn.functional.pad(W, (0, extra))[:, :N] if extra else W
+    W[:, 5] = 0
+    assert sq.sq_fold_kernel_launches(W) == 3
+    rng = np.random.default_rng(K + N)
+    s = np.exp(rng.uniform(-1, 2, K)).astype(np.float32)
+    wq, sw, gf, _ = sq.sq_fold_quant_weights(W, dev(s), g)
+    r_wq, r_sw, r_gf, _ = O.fold_quant_weights(host(W), s, host(g))
+    assert np.array_equal(host(sw), r_sw)
+    assert np.array_equal(host(wq), r_wq)
+    assert np.array_equal(host(gf), r_gf)
+
+
 @pytest.mark.parametrize("K,N", [(4096, 28672), (14336, 4096), (49152, 12288)])
 def test_fold_full_size(K, N):
     _, W, _, _ = sq_inputs.torch_case(1, K, N, 7, DEV, w_std=0.015)

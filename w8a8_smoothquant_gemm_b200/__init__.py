@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "sq_ln_smooth_quant_fp8": [P, I, I64, I64, I64, P, P, P, F, P, P, P],
             "sq_w8a8_gemm_fp8": [P, P, P, P, I64, I64, I64, P, I, I64, P, SZ, P],
             "sq_fold_next_smoothing": [P, P, I64, P, P],
+            "sq_fold_kernel_launches": [P, I, I64, I64, I64],
             "sq_alpha_search": [P, I, I64, I64, I64, P, P, F, P, I, I64, I64, P, I, P, P, SZ, P],
         }
         for name, argt in sigs.items():
@@ -243,6 +244,13 @@ def sq_ln_smooth_quant_per_tensor(x: torch.Tensor, gamma_f: torch.Tensor | None 
                                                _ptr(s), float(eps), int(static), _ptr(scale), _ptr(xq), _ptr(sx),
                                                _stream(stream)))
     return xq, sx, scale
+
+
+def sq_fold_kernel_launches(W: torch.Tensor) -> int:
+    """Kernels sq_fold_quant_weights(W, ...) launches (1, or 3 on the streaming route)."""
+    W = _mat(W, "W")
+    K, N = W.shape
+    return int(lib().sq_fold_kernel_launches(_ptr(W), _dt(W), K, N, W.stride(0)))
 
 
 def sq_w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:

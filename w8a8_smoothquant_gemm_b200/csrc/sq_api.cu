@@ -37,6 +37,7 @@ cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* w
                             int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
                             cudaStream_t st, bool* ws_too_small);
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+int fold_kernel_launches(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw);
 cudaError_t read_device_error(unsigned int* code, int clear, cudaStream_t st);
 
 namespace {
@@ -152,7 +153,7 @@ sq_status check_gemm(const void* xq, const float* sx, const void* wq, const floa
 
 extern "C" {
 
-int sq_abi_version(void) { return 101; }
+int sq_abi_version(void) { return 102; }
 
 const char* sq_status_string(sq_status status) {
   switch (status) {
@@ -258,6 +259,10 @@ sq_status sq_fold_quant_weights(const void* W, sq_dtype dt, int64_t K, int64_t N
   if (st != SQ_OK || empty) return st;
   return cuda_status(sqh::launch_fold_quant(W, dt == SQ_BF16, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f,
                                             as_stream(stream)));
+}
+
+int sq_fold_kernel_launches(const void* W, sq_dtype dt, int64_t K, int64_t N, int64_t ldw) {
+  return sqh::fold_kernel_launches(W, dt == SQ_BF16, K, N, ldw);
 }
 
 sq_status sq_ln_smooth_quant(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx, const float* gamma_f,

@@ -6,11 +6,14 @@
 //   per output channel, static; "SmoothQuant大模型平滑量化技术" demo: max/127, round, clip)
 //
 // Wq is written transposed, [N, K] with K contiguous: the GEMM's K-major operand.  Three
-// kernels cover the shapes:
-//   fold_cluster_kernel  bf16 W whose K / 16 rows per CTA fit 72 KB of shared memory: one
-//                        pass over HBM, column maxima exchanged in a thread-block cluster;
-//   fold_l2_*            taller bf16 W (large K): chunks of output channels sized to stay
-//                        in L2, a max pass then a codes pass that re-reads the chunk from L2;
+// routes cover the shapes:
+//   fold_cluster_kernel  bf16 W of at most 96 MiB whose K / 16 rows per CTA fit 72 KB of
+//                        shared memory: one pass over HBM, column maxima exchanged in a
+//                        thread-block cluster;
+//   streaming fold       larger or taller bf16 W: fold_colmax_kernel (column maxima), then
+//                        fold_codes_stream_kernel (codes of TMA-loaded tiles, last rows
+//                        first so that the part of W still in L2 is reused), then
+//                        fold_scales_kernel;
 //   fold_quant_kernel    fp32 or unaligned W: one block per strip, two passes.
 #include <algorithm>
 
@@ -267,12 +270,12 @@ __device__ __forceinline__ void fold_codes_16x4_e4m3(const uint16_t* tile, const
 // strip's scales, written to Wq transposed: item = (4 adjacent columns, 16 consecutive
 // rows); each item reads 16 x 8 bytes of shared memory and writes 16 codes to each of 4
 // rows of Wq.  F8: E4M3 codes (the FP8 variant).
-template <int CW, bool F8>
+template <int CW, bool F8, int NT = 256>
 __device__ __forceinline__ void fold_write_codes(const uint16_t* tile, const float* s_rows, const float* scale,
                                                  int64_t K, int64_t N, int RK, int64_t j0, int64_t k0,
                                                  int8_t* __restrict__ Wq) {
   const int items = (CW / 4) * (RK / 16);
-  for (int i = threadIdx.x; i < items; i += 256) {
+  for (int i = threadIdx.x; i < items; i += NT) {
     const int kq = (i % (CW / 4)) * 4, jl = (i / (CW / 4)) * 16;
     if (j0 + jl >= K) continue;  // K % 16 == 0: a 16-row block is all in or all out
     const SharedDivisor d0(scale[kq]), d1(scale[kq + 1]), d2(scale[kq + 2]), d3(scale[kq + 3]);
@@ -391,23 +394,33 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
   fold_write_codes<CW, F8>(tile, s_rows, scale, K, N, RK, j0, k0, Wq);
 }
 
-// ---------------------------------------------------------------------------- L2-blocked fold
-// Two passes over a chunk of output channels sized to stay in L2 (~40 MB of W), so W crosses
-// HBM once: pass 1 reduces max_j |s_j W_jk| of each column into sw[k] (float bits, atomicMax
-// over 256-row tiles); pass 2 re-reads the chunk (from L2), forms the scales and writes the
-// codes transposed; a last pass turns the maxima in sw into scales.  Tiles are 256 rows x 64
-// columns; no cluster or grid-wide barrier.
-template <bool BF16>
-__global__ void __launch_bounds__(256)
-fold_l2_max_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_bytes, const float* __restrict__ s,
-                   int64_t k_first, float* __restrict__ colmax, const float* __restrict__ gamma,
+// ---------------------------------------------------------------------------- two-pass fold
+// Pass 1 of the streaming fold: column maxima of |s_j W_jk| over all rows.  A block is 32
+// 16-byte column vectors x 8 row lanes; the grid covers the columns once and strides the
+// rows with four loads in flight per thread, so the loads of all blocks sweep W from the
+// first rows to the last; one atomicMax per column per block into colmax (zeroed before).
+// Also writes the folded LayerNorm vectors gamma' = gamma / s, beta' = beta / s.
+constexpr int FCM_VX = 32, FCM_RY = 8, FCM_UNROLL = 4;
+
+__device__ __forceinline__ void colmax8(float (&m)[8], const uint4 v, float sj) {
+  const float2 s2 = make_float2(sj, sj);
+  const float2 y0 = __fmul2_rn(s2, make_float2(bf16lo(v.x), bf16hi(v.x)));
+  const float2 y1 = __fmul2_rn(s2, make_float2(bf16lo(v.y), bf16hi(v.y)));
+  const float2 y2 = __fmul2_rn(s2, make_float2(bf16lo(v.z), bf16hi(v.z)));
+  const float2 y3 = __fmul2_rn(s2, make_float2(bf16lo(v.w), bf16hi(v.w)));
+  m[0] = fmaxf(m[0], fabsf(y0.x)); m[1] = fmaxf(m[1], fabsf(y0.y));
+  m[2] = fmaxf(m[2], fabsf(y1.x)); m[3] = fmaxf(m[3], fabsf(y1.y));
+  m[4] = fmaxf(m[4], fabsf(y2.x)); m[5] = fmaxf(m[5], fabsf(y2.y));
+  m[6] = fmaxf(m[6], fabsf(y3.x)); m[7] = fmaxf(m[7], fabsf(y3.y));
+}
+
+__global__ void __launch_bounds__(FCM_VX * FCM_RY)
+fold_colmax_kernel(const char* __restrict__ W, int64_t K, int64_t nvec, int64_t ldw_bytes,
+                   const float* __restrict__ s, float* __restrict__ colmax, const float* __restrict__ gamma,
                    const float* __restrict__ beta, float* __restrict__ gamma_f, float* __restrict__ beta_f) {
-  constexpr int ELT = BF16 ? 2 : 4;
-  __shared__ float red[32][64 + 1];
-  const int tid = threadIdx.x, cg = tid % 8, rl = tid / 8;
-  const int64_t k0 = k_first + (int64_t)blockIdx.x * 64 + cg * 8;
-  const int64_t j0 = (int64_t)blockIdx.y * 256;
-  if (gamma_f || beta_f) {  // the folded LayerNorm vectors, once (first chunk)
+  __shared__ float red[FCM_RY][FCM_VX * 8 + 1];
+  const int tid = threadIdx.y * FCM_VX + threadIdx.x;
+  if (gamma_f || beta_f) {
     const int64_t nb = (int64_t)gridDim.x * gridDim.y, b = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
     for (int64_t j = b * 256 + tid; j < K; j += nb * 256) {
       const float sj = s[j];
@@ -415,66 +428,97 @@ fold_l2_max_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw
       if (beta && beta_f) beta_f[j] = __fdiv_rn(beta[j], sj);
     }
   }
+  const int64_t vec = (int64_t)blockIdx.x * FCM_VX + threadIdx.x;
   float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (k0 < N) {
+  if (vec < nvec) {
+    const int64_t rstep = (int64_t)gridDim.y * FCM_RY;
+    int64_t r = (int64_t)blockIdx.y * FCM_RY + threadIdx.y;
+    const char* p = W + vec * 16;
+    for (; r + (FCM_UNROLL - 1) * rstep < K; r += FCM_UNROLL * rstep) {
+      uint4 v[FCM_UNROLL];
+      float sj[FCM_UNROLL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t j = j0 + rl + 32 * i;
-      if (j < K) {
-        float f[8];
-        const char* p = W + j * ldw_bytes + k0 * ELT;
-        if (BF16) {
-          unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(p)), f);
-        } else {
-          const float4 a = __ldg(reinterpret_cast<const float4*>(p)), c = __ldg(reinterpret_cast<const float4*>(p) + 1);
-          f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = c.x; f[5] = c.y; f[6] = c.z; f[7] = c.w;
-        }
-        const float sj = __ldg(s + j);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(__fmul_rn(sj, f[e])));
+      for (int u = 0; u < FCM_UNROLL; ++u) {
+        v[u] = ldg_stream16(p + (r + u * rstep) * ldw_bytes);
+        sj[u] = __ldg(s + r + u * rstep);
       }
+#pragma unroll
+      for (int u = 0; u < FCM_UNROLL; ++u) colmax8(m, v[u], sj[u]);
     }
+    for (; r < K; r += rstep) colmax8(m, ldg_stream16(p + r * ldw_bytes), __ldg(s + r));
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
+  for (int e = 0; e < 8; ++e) red[threadIdx.y][threadIdx.x * 8 + e] = m[e];
   __syncthreads();
-  if (tid < 64) {
-    float v = red[0][tid];
-    for (int r = 1; r < 32; ++r) v = fmaxf(v, red[r][tid]);
-    const int64_t k = k_first + (int64_t)blockIdx.x * 64 + tid;
-    if (k < N) atomic_max_nonneg(colmax + k, v);
+  const int64_t ncols = nvec * 8;
+  for (int c = tid; c < FCM_VX * 8; c += FCM_VX * FCM_RY) {
+    float v = red[0][c];
+#pragma unroll
+    for (int y = 1; y < FCM_RY; ++y) v = fmaxf(v, red[y][c]);
+    const int64_t col = (int64_t)blockIdx.x * FCM_VX * 8 + c;
+    if (col < ncols) atomic_max_nonneg(colmax + col, v);
   }
 }
 
-// Pass 2 (bf16 weights): the 256 x 64 tile (from L2) into shared memory, scales from the
-// column maxima, codes written transposed (fold_write_codes).  F8: E4M3 codes, max / 448.
-template <bool F8>
-__global__ void __launch_bounds__(256)
-fold_l2_codes_kernel(const char* __restrict__ W, int64_t K, int64_t N, int64_t ldw_bytes, const float* __restrict__ s,
-                     int64_t k_first, const float* __restrict__ colmax, int8_t* __restrict__ Wq) {
-  __shared__ __align__(16) uint16_t tile[256 * 64];  // W[j0 + r, kt + c] bf16 bits at r * 64 + c
-  __shared__ float s_rows[256];
-  __shared__ float scale[64];
-  const int tid = threadIdx.x, cg = tid % 8, rl = tid / 8;
-  const int64_t kt = k_first + (int64_t)blockIdx.x * 64;
-  const int64_t j0 = (int64_t)blockIdx.y * 256;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = rl + 32 * i;
-    const int64_t j = j0 + r, k = kt + cg * 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < K && k < N) v = __ldg(reinterpret_cast<const uint4*>(W + j * ldw_bytes + k * 2));
-    *reinterpret_cast<uint4*>(tile + r * 64 + cg * 8) = v;
+// Pass 2: the codes of RT-row x 64-column tiles of W (RT threads, one 16-row x 4-column item
+// each), written transposed into Wq (fold_write_codes).  Persistent blocks walk the tiles
+// with the last rows first: pass 1 read those last, so the part of W still in L2 is read
+// from there.  One thread TMA-loads each tile into an S-stage shared-memory ring, S - 1
+// tiles ahead of the block's codes.
+constexpr int FCS_CW = 64;
+
+template <int RT, int S, bool F8>
+__global__ void __launch_bounds__(RT, 896 / RT)  // 7 blocks of 128 threads per SM (72 registers)
+fold_codes_stream_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t N,
+                         const float* __restrict__ s, const float* __restrict__ colmax, int8_t* __restrict__ Wq,
+                         unsigned int* err) {
+  constexpr uint32_t TILE = RT * FCS_CW * 2;
+  static_assert(RT >= FCS_CW && (FCS_CW / 4) * (RT / 16) == RT, "one item per thread");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ float s_rows[RT];
+  __shared__ float scale[FCS_CW];
+  __shared__ __align__(8) uint64_t bars[S];
+  const int tid = threadIdx.x;
+  const int64_t strips = (N + FCS_CW - 1) / FCS_CW, rtiles = (K + RT - 1) / RT;
+  const int64_t units = strips * rtiles;
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  auto row0 = [&](int64_t u) { return (rtiles - 1 - u / strips) * RT; };
+  auto col0 = [&](int64_t u) { return (u % strips) * FCS_CW; };
+  auto issue = [&](int64_t u, int stage) {
+    const uint32_t b = smem_u32(&bars[stage]);
+    mbar_arrive_expect_tx(b, TILE);
+    tma_load_2d(smem_u32(ring + (size_t)stage * TILE), &wmap, b, (int)col0(u), (int)row0(u));
+  };
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  s_rows[tid] = (j0 + tid < K) ? __ldg(s + j0 + tid) : 0.0f;
-  if (tid < 64) scale[tid] = (kt + tid < N) ? __fdiv_rn(__ldg(colmax + kt + tid), F8 ? 448.0f : 127.0f) : 0.0f;
   __syncthreads();
-  fold_write_codes<64, F8>(tile, s_rows, scale, K, N, 256, j0, kt, Wq);
+  if (tid == 0)
+    for (int i = 0; i < S - 1 && first + i * step < units; ++i) issue(first + i * step, i);
+  for (int64_t i = 0; first + i * step < units; ++i) {
+    const int64_t u = first + i * step;
+    const int64_t j0 = row0(u), k0 = col0(u);
+    // the stage of tile i + S - 1 held tile i - 1, whose reads ended at the previous barrier
+    if (tid == 0 && u + (S - 1) * step < units) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(u + (S - 1) * step, (int)((i + S - 1) % S));
+    }
+    s_rows[tid] = (j0 + tid < K) ? __ldg(s + j0 + tid) : 0.0f;
+    if (tid < FCS_CW) scale[tid] = (k0 + tid < N) ? __fdiv_rn(__ldg(colmax + k0 + tid), F8 ? 448.0f : 127.0f) : 0.0f;
+    __syncthreads();
+    const int stage = (int)(i % S);
+    if (!mbar_wait(smem_u32(&bars[stage]), (uint32_t)((i / S) & 1))) atomicOr(err, ERR_FOLD_TMA_WAIT);
+    fold_write_codes<FCS_CW, F8, RT>(reinterpret_cast<const uint16_t*>(ring + (size_t)stage * TILE), s_rows, scale,
+                                     K, N, RT, j0, k0, Wq);
+    __syncthreads();
+  }
 }
 
 // sw[k] = RN(max_k / 127) (F8: / 448) in place.
 template <bool F8>
-__global__ void fold_l2_scales_kernel(float* __restrict__ sw, int64_t N) {
+__global__ void fold_scales_kernel(float* __restrict__ sw, int64_t N) {
   const int64_t k = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (k < N) sw[k] = __fdiv_rn(sw[k], F8 ? 448.0f : 127.0f);
 }
@@ -563,53 +607,93 @@ static bool fold_cluster_shape(int64_t K, size_t budget, int* cw, int* c, int* r
   return false;
 }
 
-// L2-blocked two-pass fold of bf16 weights: chunks of output channels whose W columns fit
-// ~40 MB, each a max pass then a codes pass (which reads the chunk again from L2).
-template <bool F8>
-static cudaError_t launch_fold_l2(const void* W, int64_t K, int64_t N, int64_t ldw, const float* s,
-                                  const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
-                                  float* beta_f, cudaStream_t st) {
+// Streaming two-pass fold of bf16 weights: column maxima into sw, the codes pass (RT-row
+// tiles in an S-stage TMA ring, as many blocks as fit on the SMs), then the maxima in sw
+// become scales.
+template <int RT, int S, bool F8>
+static cudaError_t launch_fold_stream(const void* W, int64_t K, int64_t N, int64_t ldw, const float* s,
+                                      const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
+                                      float* beta_f, cudaStream_t st) {
+  CUtensorMap map;
+  if (!make_tmap_2d(&map, true, W, N, K, ldw * 2, sqk::FCS_CW, RT, false)) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(sw, 0, sizeof(float) * (size_t)N, st);
   if (e != cudaSuccess) return e;
-  const int64_t ldb = ldw * 2;
-  int64_t chunk = (int64_t)(40ll << 20) / (K * 2) / 64 * 64;
-  chunk = std::max<int64_t>(64, std::min<int64_t>(chunk, (N + 63) / 64 * 64));
-  const unsigned rows = (unsigned)((K + 255) / 256);
-  for (int64_t k0 = 0; k0 < N; k0 += chunk) {
-    const int64_t kc = std::min<int64_t>(chunk, N - k0);
-    const dim3 grid((unsigned)((kc + 63) / 64), rows);
-    const bool first = k0 == 0;
-    sqk::fold_l2_max_kernel<true><<<grid, 256, 0, st>>>((const char*)W, K, N, ldb, s, k0, sw, gamma, beta,
-                                                         first ? gamma_f : nullptr, first ? beta_f : nullptr);
-    sqk::fold_l2_codes_kernel<F8><<<grid, 256, 0, st>>>((const char*)W, K, N, ldb, s, k0, sw, Wq);
-  }
-  sqk::fold_l2_scales_kernel<F8><<<(unsigned)((N + 255) / 256), 256, 0, st>>>(sw, N);
+  const int64_t nvec = N / 8;
+  const int64_t gx = (nvec + sqk::FCM_VX - 1) / sqk::FCM_VX;
+  // one wave: as many blocks as are resident at once (44 registers: 5 per SM), each
+  // striding over the rows; measured 114 against 119 us at 4096 x 28672 over 8 per SM
+  int occ = 1;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, sqk::fold_colmax_kernel, sqk::FCM_VX * sqk::FCM_RY, 0);
+  if (e != cudaSuccess) return e;
+  int64_t gy = std::max<int64_t>(1, (int64_t)num_sms() * std::max(occ, 1) / gx);
+  gy = std::min<int64_t>(gy, (K + sqk::FCM_RY - 1) / sqk::FCM_RY);
+  gy = std::min<int64_t>(gy, 65535);
+  sqk::fold_colmax_kernel<<<dim3((unsigned)gx, (unsigned)gy), dim3(sqk::FCM_VX, sqk::FCM_RY), 0, st>>>(
+      (const char*)W, K, nvec, ldw * 2, s, sw, gamma, beta, gamma_f, beta_f);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kern = sqk::fold_codes_stream_kernel<RT, S, F8>;
+  const size_t smem = 128 + (size_t)S * RT * sqk::FCS_CW * 2;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 1;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, RT, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t units = (N + sqk::FCS_CW - 1) / sqk::FCS_CW * ((K + RT - 1) / RT);
+  const int64_t grid = std::min<int64_t>(units, (int64_t)num_sms() * std::max(per_sm, 1));
+  kern<<<(unsigned)grid, RT, smem, st>>>(map, K, N, s, sw, Wq, error_word_ptr());
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sqk::fold_scales_kernel<F8><<<(unsigned)((N + 255) / 256), 256, 0, st>>>(sw, N);
   return cudaGetLastError();
+}
+
+// Route of a fold: the one-shot cluster fold for bf16 W of at most 96 MiB whose cluster
+// block fits; the streaming fold for other 16-byte-aligned bf16 W; the strip kernel
+// otherwise.  Measured on W 4096 x {4096, 6144, 28672} and 14336 x 4096: the cluster fold
+// leads below ~100 MB of W (23 against 25 us at 4096 x 4096), the streaming fold above
+// (111 against 124 us at 4096 x 28672, 60 against 75 us at 14336 x 4096).
+enum FoldRoute { FOLD_CLUSTER, FOLD_STREAM, FOLD_STRIPS };
+
+static FoldRoute fold_route(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, int* cw, int* cl, int* rk) {
+  const bool tma_ok = bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && (ldw * 2) % 16 == 0;
+  if (!tma_ok) return FOLD_STRIPS;
+  if (K * N * 2 <= (96ll << 20) && fold_cluster_shape(K, 72 * 1024, cw, cl, rk)) return FOLD_CLUSTER;
+  return FOLD_STREAM;
+}
+
+int fold_kernel_launches(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw) {
+  if (K <= 0 || N <= 0) return 0;
+  int cw = 0, cl = 0, rk = 0;
+  return fold_route(W, bf16, K, N, ldw, &cw, &cl, &rk) == FOLD_STREAM ? 3 : 1;
 }
 
 template <bool F8>
 static cudaError_t launch_fold_any(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
-                              const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
-                              float* beta_f, cudaStream_t st) {
+                                   const float* gamma, const float* beta, int8_t* Wq, float* sw, float* gamma_f,
+                                   float* beta_f, cudaStream_t st) {
   int cw = 0, cl = 0, rk = 0;
-  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && fold_cluster_shape(K, 72 * 1024, &cw, &cl, &rk)) {
-    switch (cw) {
-      case 64: return launch_fold_cluster_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-      case 32: return launch_fold_cluster_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-      default: return launch_fold_cluster_t<16, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
-    }
+  switch (fold_route(W, bf16, K, N, ldw, &cw, &cl, &rk)) {
+    case FOLD_CLUSTER:
+      switch (cw) {
+        case 64: return launch_fold_cluster_t<64, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+        case 32: return launch_fold_cluster_t<32, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+        default: return launch_fold_cluster_t<16, F8>(W, K, N, ldw, cl, rk, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+      }
+    case FOLD_STREAM:
+      // 128-row tiles, one stage: seven 4-warp blocks per SM measured faster than deeper
+      // rings with fewer blocks (111 against 125 us for 256-row tiles in a 2-stage ring)
+      return launch_fold_stream<128, 1, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+    default: break;
   }
-  // blocks too tall for the one-shot fold (large K): the L2-blocked two-pass fold
-  if (bf16 && (reinterpret_cast<uintptr_t>(W) % 16) == 0 && (ldw * 2) % 16 == 0)
-    return launch_fold_l2<F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
   // narrower strips when there are few output channels, so every SM gets work
   const int64_t sms = num_sms();
   const int strip = (N / 32 >= 2 * sms) ? 32 : 16;
   if (bf16)
     return strip == 32 ? launch_fold_t<true, 32, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
-                    : launch_fold_t<true, 16, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+                       : launch_fold_t<true, 16, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
   return strip == 32 ? launch_fold_t<false, 32, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st)
-                  : launch_fold_t<false, 16, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
+                     : launch_fold_t<false, 16, F8>(W, K, N, ldw, s, gamma, beta, Wq, sw, gamma_f, beta_f, st);
 }
 
 cudaError_t launch_fold_quant(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
