@@ -225,35 +225,44 @@ class Linear:
 
 
 def quantizer_profile(sq, layers, world, reps=5) -> dict:
-    """Per-kernel CUDA-event times of the bandwidth kernels (separate from the timed steps)."""
+    """Per-kernel CUDA-event times of the bandwidth kernels (separate from the timed steps).
+
+    Before each timed kernel a 256 MB buffer is zeroed on the same stream: the L2 starts cold,
+    and the device is still busy with it when the host has enqueued the kernel and its closing
+    event, so an interval holds the kernel's device time, not the host's launch latency."""
     kinds = ("calib", "wabsmax", "fold", "quant")
     tot = {k: 0.0 for k in kinds}
     byt = {k: 0 for k in kinds}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=layers[0].x.device)
+    pending = []
+
+    def timed(kind, nbytes, fn):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        pending.append((kind, nbytes, a, b))
+
     for _ in range(reps):
         for L in layers:
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-            ev[0].record()
             if L.ln:
-                sq.sq_calib_ln_absmax(L.x, L.gamma, out=L.ax)
+                timed("calib", L.bytes_calib(), lambda: sq.sq_calib_ln_absmax(L.x, L.gamma, out=L.ax))
             else:
-                sq.sq_calib_absmax(L.x, 0, out=L.ax)
-            ev[1].record()
-            sq.sq_calib_absmax(L.W, 1, out=L.aw)
-            ev[2].record()
+                timed("calib", L.bytes_calib(), lambda: sq.sq_calib_absmax(L.x, 0, out=L.ax))
+            timed("wabsmax", L.bytes_wabsmax(), lambda: sq.sq_calib_absmax(L.W, 1, out=L.aw))
             sq.sq_smooth_factors(L.ax, L.aw, ALPHA, out=L.s)
-            ev[3].record()
-            sq.sq_fold_quant_weights(L.W, L.s, L.gamma if L.ln else None, wq=L.wq, sw=L.sw, gamma_f=L.gf)
-            ev[4].record()
+            timed("fold", L.bytes_fold(),
+                  lambda: sq.sq_fold_quant_weights(L.W, L.s, L.gamma if L.ln else None, wq=L.wq, sw=L.sw,
+                                                   gamma_f=L.gf))
             if L.ln:
-                sq.sq_ln_smooth_quant(L.x, gamma_f=L.gf, xq=L.xq, sx=L.sx)
+                timed("quant", L.bytes_quant(), lambda: sq.sq_ln_smooth_quant(L.x, gamma_f=L.gf, xq=L.xq, sx=L.sx))
             else:
-                sq.sq_ln_smooth_quant(L.x, s=L.s, xq=L.xq, sx=L.sx)
-            ev[5].record()
-            torch.cuda.synchronize()
-            for k, (a, b), nb in zip(kinds, ((0, 1), (1, 2), (3, 4), (4, 5)),
-                                     (L.bytes_calib(), L.bytes_wabsmax(), L.bytes_fold(), L.bytes_quant())):
-                tot[k] += ev[a].elapsed_time(ev[b]) / 1e3
-                byt[k] += nb
+                timed("quant", L.bytes_quant(), lambda: sq.sq_ln_smooth_quant(L.x, s=L.s, xq=L.xq, sx=L.sx))
+    torch.cuda.synchronize()
+    for kind, nbytes, a, b in pending:
+        tot[kind] += a.elapsed_time(b) / 1e3
+        byt[kind] += nbytes
     return {f"{k}_gbs": round(byt[k] / tot[k] / 1e9, 1) for k in kinds}
 
 
