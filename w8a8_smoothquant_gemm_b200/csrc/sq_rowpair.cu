@@ -493,8 +493,8 @@ static cudaError_t launch_rowpair(const void* x, int64_t M, int64_t ld_bytes, co
 
 // Row lengths with a chunk-pair kernel (bf16 rows only).  Quantisers: K in {512, 1024, 2048,
 // 4096, 8192, 12288, 14336}; calibration (whose running maxima also live in registers):
-// K in {512, 1024, 2048, 4096, 8192}.  Below `min_rows` rows the per-row latency of a
-// one-warp row outweighs its instruction savings and the staged kernel is used instead.
+// K in {512, 1024, 2048, 4096, 8192}.  Below 1024 rows the staged kernel of sq_rowpipe.cu
+// runs instead: with few rows per group, the per-row latency outweighs the instruction savings.
 bool rowpair_supported(int64_t K, bool bf16, bool calib, int64_t rows) {
   if (!bf16 || rows < 1024) return false;
   switch (K) {
