@@ -149,10 +149,11 @@ def test_fold_quant_weights(dt, K, N, extra):
     assert np.array_equal(host(gf), r[2]) and np.array_equal(host(bf), r[3])
 
 
-@pytest.mark.parametrize("K,N,extra", [(40000, 1288, 8), (49168, 1096, 0)])
+@pytest.mark.parametrize("K,N,extra", [(40000, 1288, 8), (49168, 1096, 0), (16, 3145800, 0)])
 def test_fold_streaming_ragged(K, N, extra):
     """The streaming two-pass route on a ragged last row tile and column strip, with a padded
-    leading dimension and an all-zero output channel."""
+    leading dimension and an all-zero output channel; K = 16 is a single, mostly empty row
+    tile under a 100 MB wide weight."""
     _, W, g, _ = sq_inputs.torch_case(1, K, N, 11, DEV, w_std=0.015)
     W = torch.nn.functional.pad(W, (0, extra))[:, :N] if extra else W
     W[:, 5] = 0
