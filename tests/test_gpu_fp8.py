@@ -59,6 +59,23 @@ def test_fold_fp8(dt, K, N):
     assert np.array_equal(host(gf), r_gf)
 
 
+def test_fold_fp8_streaming_padded():
+    """E4M3 codes on the streaming two-pass route with a padded leading dimension (ragged last
+    row tile and column strip, a zero column, -0 entries)."""
+    K, N, extra = 40016, 1288, 8
+    _, W, g, _ = sq_inputs.torch_case(1, K, N, 13, DEV, w_std=0.015)
+    W = torch.nn.functional.pad(W, (0, extra))[:, :N]
+    W[:, 3] = 0
+    W[::5, 6] = -0.0
+    assert sq.sq_fold_kernel_launches(W) == 3
+    s = np.exp(np.random.default_rng(K).uniform(-1, 1.5, K)).astype(np.float32)
+    wq, sw, gf, _ = sq.sq_fold_quant_weights_fp8(W, dev(s), g)
+    r_wq, r_sw, r_gf, _ = O.fold_quant_weights_fp8(host(W), s, host(g))
+    assert np.array_equal(host(sw), r_sw)
+    assert np.array_equal(host(wq), r_wq)
+    assert np.array_equal(host(gf), r_gf)
+
+
 # ----------------------------------------------------------------------------- per-token quantiser
 @pytest.mark.parametrize("M,K", [(1, 16), (5, 256), (33, 2048), (64, 4096), (3, 16400), (2, 49152),
                                  (1031, 4096), (1029, 14336), (1030, 512), (1030, 12288), (1100, 8192)])
