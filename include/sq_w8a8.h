@@ -188,7 +188,8 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *   SQ_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads the
  *   library holds until the process exits.  The caller still passes all inputs and
  *   outputs, with the same meaning, layout and checks as sq_w8a8_gemm.
- *   - A shape whose workspace (sq_w8a8_gemm_workspace_size) exceeds the scratch returns
+ *   - The arguments are checked first, in the order sq_w8a8_gemm checks them; then a shape
+ *     whose workspace (sq_w8a8_gemm_workspace_size) exceeds the scratch returns
  *     SQ_ERR_WORKSPACE with nothing launched.
  *   - The first call on a device looks up the scratch array's device address (set-up, once
  *     per device, with that device current); make that first call before any stream
@@ -270,6 +271,22 @@ sq_status sq_w8a8_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq
 /* Reads (and with clear != 0 resets) the device-side error word of the current device:
  * 0 when no kernel gave up on a bounded wait.  Synchronises `stream`. */
 sq_status sq_device_error(unsigned int* code, int clear, void* stream);
+
+/* sq_selfcheck_shared_divisor -- checks, on the device, the division every quantiser and the
+ * weight fold use for code = rne(v / scale) ("SmoothQuant大模型平滑量化技术", Python demo: the code
+ * is the rounded quotient, so the quotient must be the correctly rounded one).  The kernels
+ * divide all elements of a row (column) by one shared scale through one correctly rounded
+ * reciprocal and Markstein's correction step; this call evaluates that routine, in its scalar
+ * and its packed-pair form, on every pair (a[j], b[i]) and compares the bits with IEEE
+ * round-to-nearest division:
+ *   counts[0] += pairs where the scalar form differs, counts[1] += where the packed form
+ *   differs, counts[2] += pairs checked (zero divisors are skipped: a zero scale means
+ *   "all codes 0" and has no quotient).
+ *   a: fp32 [na] dividends, na even, 2 <= na <= 4096; b: fp32 [nb] divisors; q: NULL or fp32
+ *   [nb, na], the scalar form's quotients (q[i * na + j] = a[j] / b[i]); counts: 3 device
+ *   uint64, 8-byte aligned, accumulated into (zero them first).  All device pointers. */
+sq_status sq_selfcheck_shared_divisor(const float* a, int64_t na, const float* b, int64_t nb, float* q,
+                                      unsigned long long* counts, void* stream);
 
 /* Human-readable name of a status. */
 const char* sq_status_string(sq_status status);

@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.sqo_f32_to_bf16.restype = ctypes.c_uint16
         L.sqo_num_threads.argtypes = []
         L.sqo_num_threads.restype = I
+        L.sqo_set_num_threads.argtypes = [I]
+        L.sqo_set_num_threads.restype = None
         _lib = L
     return _lib
 
@@ -79,6 +81,11 @@ def lib() -> ctypes.CDLL:
 def num_threads() -> int:
     """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS or all cores)."""
     return lib().sqo_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the oracle's following parallel loops (results do not depend on it)."""
+    lib().sqo_set_num_threads(int(n))
 
 
 def _ptr(a):

@@ -62,6 +62,16 @@ int sqo_num_threads(void) {
 #endif
 }
 
+/* Threads for the following parallel loops (timing only: every result is row- or
+ * column-parallel and identical for any thread count). */
+void sqo_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* bfloat16 is the top half of a binary32; widening is exact. */
 static float bf16_to_f32(uint16_t h) {
   uint32_t u = (uint32_t)h << 16;

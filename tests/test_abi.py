@@ -145,6 +145,26 @@ def test_gemm_validation():
     assert call(M=0) == 0 and call(N=0, ldy=0) == 0
 
 
+def test_gemm_noalloc_checks_arguments_before_its_scratch_size():
+    """The no-allocation GEMM reports a bad argument as sq_w8a8_gemm does, even for a shape whose
+    workspace would not fit its built-in scratch (which is checked only after the arguments)."""
+    f = sq.lib().sq_w8a8_gemm_noalloc
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    f.argtypes = [P, P, P, P, I64, I64, I64, P, I, I64, P]
+    f.restype = I
+
+    def call(xq=A16, sx=A16b, wq=A16c, sw=A16b, M=96, N=1 << 20, K=65536, y=A16, ydt=BF16, ldy=1 << 20):
+        return f(xq, sx, wq, sw, M, N, K, y, ydt, ldy, NULL)
+
+    assert call(xq=NULL) == INVALID
+    assert call(sx=NULL) == INVALID
+    assert call(K=40) == ALIGN
+    assert call(y=ctypes.c_void_p(0x10001)) == ALIGN
+    assert call(K=SQ_MAX_K_PLUS) == UNSUPPORTED
+    assert call(ldy=16) == INVALID
+    assert call(M=0) == 0
+
+
 def test_workspace_size_validation():
     f = sq.lib().sq_w8a8_gemm_workspace_size
     assert f(4, 4, 0) == ctypes.c_size_t(-1).value

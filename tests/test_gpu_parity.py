@@ -283,7 +283,8 @@ def test_per_tensor_many_rows(K, mode):
     assert (np.abs(r_xq) == 127).sum() > 0
 
 
-@pytest.mark.parametrize("rows,K", [(1030, 512), (1100, 1024), (1027, 2048), (2051, 4096), (1500, 8192)])
+@pytest.mark.parametrize("rows,K", [(1030, 512), (1100, 1024), (1027, 2048), (2051, 4096), (1500, 8192),
+                                    (2048, 12288), (2051, 14336)])
 def test_calib_ln_absmax_many_rows(rows, K):
     c = _many_rows(rows, K, rows + 3 * K)
     x = dev(padded(c.x, 8))[:, :K]
@@ -390,24 +391,36 @@ def test_decode_layer_full(M, K, N, ln):
 
 
 SAMPLED = [(8192, 4096, 28672, True, 0.02), (2048, 14336, 4096, False, 0.02), (2048, 4096, 6144, True, 0.02),
-           (2048, 12288, 49152, True, 0.015), (16, 49152, 12288, False, 0.015)]
+           (2048, 12288, 36864, True, 0.015), (2048, 12288, 12288, False, 0.015),
+           (2048, 12288, 49152, True, 0.015), (2048, 49152, 12288, False, 0.015), (16, 49152, 12288, False, 0.015)]
 
 
 @pytest.mark.parametrize("M,K,N,ln,w_std", SAMPLED)
 def test_large_layer_sampled_rows(M, K, N, ln, w_std):
-    """Full-size prefill / 175B-class shapes: statistics, codes and scales compared in full on the
-    quantities the oracle computes quickly; the GEMM on sampled rows (all N columns)."""
+    """Full-size prefill and 175B-class linears, calibrated on their own batch.  The statistics
+    (activation absmax over all M rows, of LN(x) where a LayerNorm precedes; weight absmax), the
+    smoothing factors, the folded LayerNorm weight, every weight code and every weight scale are
+    compared with the oracle in full, bit for bit.  The per-token codes and scales, and the GEMM
+    output, on sampled rows (every column of those rows) from the oracle's own chain."""
     g = _layer(M, K, N, 200 + M + N, w_std, ln)
+    ax = O.calib_ln_absmax(g["x"], g["gamma"]) if ln else O.calib_absmax(g["x"], 0)
+    assert np.array_equal(g["ax"], ax)
     aw = O.calib_absmax(g["W"], 1)
     assert np.array_equal(g["aw"], aw)
-    rows = np.unique(np.concatenate([np.linspace(0, M - 1, 6).astype(int), [M - 1]]))
-    # per-token codes of the sampled rows from the GPU's own statistics
+    s = O.smooth_factors(ax, aw, 0.5)
+    assert np.array_equal(g["s"], s)
+    wq, sw, gf, _ = O.fold_quant_weights(g["W"], s, g["gamma"] if ln else None)
+    assert np.array_equal(g["sw"], sw)
+    assert np.array_equal(g["wq"], wq)
     if ln:
-        xq, sx = O.ln_smooth_quant(g["x"][rows], gamma_f=g["gf"])
+        assert np.array_equal(g["gf"], gf)
+    rows = np.unique(np.concatenate([np.linspace(0, M - 1, 6).astype(int), [M - 1]]))
+    if ln:
+        xq, sx = O.ln_smooth_quant(g["x"][rows], gamma_f=gf)
     else:
-        xq, sx = O.ln_smooth_quant(g["x"][rows], s=g["s"])
+        xq, sx = O.ln_smooth_quant(g["x"][rows], s=s)
     assert np.array_equal(g["xq"][rows], xq) and np.array_equal(g["sx"][rows], sx)
-    ref = O.w8a8_gemm(xq, sx, g["wq"], g["sw"], "bf16")
+    ref = O.w8a8_gemm(xq, sx, wq, sw, "bf16")
     assert assert_bf16_close(g["y"][rows], ref) == 1.0
 
 

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "sq_fold_next_smoothing": [P, P, I64, P, P],
             "sq_fold_kernel_launches": [P, I, I64, I64, I64],
             "sq_alpha_search": [P, I, I64, I64, I64, P, P, F, P, I, I64, I64, P, I, P, P, SZ, P],
+            "sq_selfcheck_shared_divisor": [P, I64, P, I64, P, P, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -390,6 +391,19 @@ def sq_w8a8_gemm_fp8(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: t
     _check("sq_w8a8_gemm_fp8", lib().sq_w8a8_gemm_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
                                                       y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))
     return y
+
+
+def sq_selfcheck_shared_divisor(a: torch.Tensor, b: torch.Tensor, want_quotients: bool = False, stream=None):
+    """Checks the library's shared-divisor quotient against IEEE division for every pair
+    (a[j], b[i]).  Returns ([scalar mismatches, packed mismatches, pairs checked] as a CUDA int64
+    tensor, quotients [nb, na] or None)."""
+    _vec(a, a.numel(), "a")
+    _vec(b, b.numel(), "b")
+    counts = torch.zeros(3, dtype=torch.int64, device=a.device)
+    q = torch.empty(b.numel(), a.numel(), dtype=torch.float32, device=a.device) if want_quotients else None
+    _check("sq_selfcheck_shared_divisor", lib().sq_selfcheck_shared_divisor(_ptr(a), a.numel(), _ptr(b), b.numel(),
+                                                                            _ptr(q), _ptr(counts), _stream(stream)))
+    return counts, q
 
 
 def sq_device_error(clear: bool = True, stream=None) -> int:

@@ -151,6 +151,15 @@ sq_status check_gemm(const void* xq, const float* sx, const void* wq, const floa
 }
 }  // namespace
 
+namespace sqh {
+// The argument checks of sq_w8a8_gemm (for entry points that wrap it); *empty is set when the
+// shape is empty and nothing is to be launched.
+sq_status check_gemm_args(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
+                          int64_t K, const void* y, sq_dtype ydt, int64_t ldy, bool* empty) {
+  return check_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, nullptr, true, empty);
+}
+}  // namespace sqh
+
 extern "C" {
 
 int sq_abi_version(void) { return 102; }

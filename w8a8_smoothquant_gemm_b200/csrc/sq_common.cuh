@@ -74,6 +74,15 @@ struct SharedDivisor {
   }
 };
 
+// The same quotient on a packed binary32 pair, each half with its own divisor: rc holds the
+// two correctly rounded reciprocals, nb the two negated divisors.  Each half rounds exactly as
+// SharedDivisor::div_fast does.
+__device__ __forceinline__ float2 markstein2(float2 a, float2 rc, float2 nb) {
+  const float2 q = __fmul2_rn(a, rc);
+  const float2 r = __ffma2_rn(q, nb, a);
+  return __ffma2_rn(r, rc, q);
+}
+
 // Code of v with a shared scale, returned in the low byte of a 32-bit word: the
 // correctly rounded quotient q = v / scale satisfies |q| <= 127 (1 + 2^-23) because
 // |v| <= absmax and scale = RN(absmax / 127), so adding 1.5 * 2^23 rounds q to the nearest
@@ -104,10 +113,7 @@ __device__ __forceinline__ uint2 pack8_codes(const float* y, const SharedDivisor
     const float2 magic = make_float2(12582912.0f, 12582912.0f);
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
-      const float2 a = make_float2(y[e], y[e + 1]);
-      const float2 q = __fmul2_rn(a, rc);
-      const float2 r = __ffma2_rn(q, nb, a);
-      float2 qq = __ffma2_rn(r, rc, q);
+      float2 qq = markstein2(make_float2(y[e], y[e + 1]), rc, nb);
       if (CLAMP) qq = make_float2(fminf(fmaxf(qq.x, -127.0f), 127.0f), fminf(fmaxf(qq.y, -127.0f), 127.0f));
       const float2 t = __fadd2_rn(qq, magic);
       c[e] = __float_as_uint(t.x);
@@ -163,10 +169,7 @@ __device__ __forceinline__ uint2 pack8_e4m3(const float* y, const SharedDivisor&
     const float2 rc = make_float2(d.y, d.y), nb = make_float2(-d.b, -d.b);
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
-      const float2 a = make_float2(y[e], y[e + 1]);
-      const float2 q0 = __fmul2_rn(a, rc);
-      const float2 r = __ffma2_rn(q0, nb, a);
-      const float2 qq = __ffma2_rn(r, rc, q0);
+      const float2 qq = markstein2(make_float2(y[e], y[e + 1]), rc, nb);
       q[e] = with_sign_of(qq.x, y[e]);
       q[e + 1] = with_sign_of(qq.y, y[e + 1]);
     }

@@ -204,10 +204,8 @@ __device__ __forceinline__ void fold_codes_16x4(const uint16_t* tile, const floa
       const float2 y01 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.x), bf16hi(w.x)));
       const float2 y23 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.y), bf16hi(w.y)));
       if (FAST) {
-        const float2 q01 = __fmul2_rn(y01, rc01), q23 = __fmul2_rn(y23, rc23);
-        const float2 e01 = __ffma2_rn(q01, nb01, y01), e23 = __ffma2_rn(q23, nb23, y23);
-        const float2 t01 = __fadd2_rn(__ffma2_rn(e01, rc01, q01), magic);
-        const float2 t23 = __fadd2_rn(__ffma2_rn(e23, rc23, q23), magic);
+        const float2 t01 = __fadd2_rn(markstein2(y01, rc01, nb01), magic);
+        const float2 t23 = __fadd2_rn(markstein2(y23, rc23, nb23), magic);
         b[0][r] = __float_as_uint(t01.x);
         b[1][r] = __float_as_uint(t01.y);
         b[2][r] = __float_as_uint(t23.x);
@@ -247,9 +245,8 @@ __device__ __forceinline__ void fold_codes_16x4_e4m3(const uint16_t* tile, const
       const float2 y01 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.x), bf16hi(w.x)));
       const float2 y23 = __fmul2_rn(make_float2(sj, sj), make_float2(bf16lo(w.y), bf16hi(w.y)));
       if (FAST) {
-        const float2 q01 = __fmul2_rn(y01, rc01), q23 = __fmul2_rn(y23, rc23);
-        const float2 t01 = __ffma2_rn(__ffma2_rn(q01, nb01, y01), rc01, q01);
-        const float2 t23 = __ffma2_rn(__ffma2_rn(q23, nb23, y23), rc23, q23);
+        const float2 t01 = markstein2(y01, rc01, nb01);
+        const float2 t23 = markstein2(y23, rc23, nb23);
         q[0][r] = with_sign_of(t01.x, y01.x);
         q[1][r] = with_sign_of(t01.y, y01.y);
         q[2][r] = with_sign_of(t23.x, y23.x);

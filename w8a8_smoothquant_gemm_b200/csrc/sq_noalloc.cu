@@ -18,7 +18,8 @@
 #include "sq_common.cuh"
 
 namespace sqh {
-size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+sq_status check_gemm_args(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
+                          int64_t K, const void* y, sq_dtype ydt, int64_t ldy, bool* empty);
 }
 
 namespace {
@@ -51,9 +52,12 @@ cudaError_t scratch_address(void** addr) {
 extern "C" sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                                           int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                                           void* stream) {
+  // the same argument checks, in the same order, as sq_w8a8_gemm; the scratch size comes after
+  bool empty = false;
+  const sq_status st = sqh::check_gemm_args(xq, sx, wq, sw, M, N, K, y, ydt, ldy, &empty);
+  if (st != SQ_OK || empty) return st;
   const size_t need = sq_w8a8_gemm_workspace_size(M, N, K);
-  if (need == (size_t)-1 || need == 0)  // invalid sizes are reported by the checks of sq_w8a8_gemm
-    return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, nullptr, 0, stream);
+  if (need == 0) return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, nullptr, 0, stream);
   if (need > (size_t)SQ_NOALLOC_SCRATCH_BYTES) return SQ_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return SQ_ERR_CUDA;

@@ -144,8 +144,7 @@ __device__ __forceinline__ void pair_codes_e4m3(const float2* v, const SharedDiv
     const float2 rc = make_float2(d.y, d.y), nb = make_float2(-d.b, -d.b);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float2 q = __fmul2_rn(v[e], rc);
-      const float2 qq = __ffma2_rn(__ffma2_rn(q, nb, v[e]), rc, q);
+      const float2 qq = markstein2(v[e], rc, nb);
       lo[e] = with_sign_of(qq.x, v[e].x);
       hi[e] = with_sign_of(qq.y, v[e].y);
     }
@@ -169,9 +168,7 @@ __device__ __forceinline__ void pair_codes_fast(const float2* v, const SharedDiv
   uint32_t lo[8], hi[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    const float2 q = __fmul2_rn(v[e], rc);
-    const float2 r = __ffma2_rn(q, nb, v[e]);
-    float2 qq = __ffma2_rn(r, rc, q);
+    float2 qq = markstein2(v[e], rc, nb);
     if (CLAMP) qq = make_float2(fminf(fmaxf(qq.x, -127.0f), 127.0f), fminf(fmaxf(qq.y, -127.0f), 127.0f));
     const float2 s = __fadd2_rn(qq, magic);
     lo[e] = __float_as_uint(s.x);
@@ -350,11 +347,8 @@ rowpair_kernel(const char* __restrict__ x, int64_t M, int64_t ld_bytes, const fl
           const float4 rs = vb[h * NPAIR + q * T + t];
           const float2 r01 = make_float2(rs.x, rs.y), r23 = make_float2(rs.z, rs.w);
           const float2 x01 = v[q][2 * h], x23 = v[q][2 * h + 1];
-          const float2 q01 = __fmul2_rn(x01, r01), q23 = __fmul2_rn(x23, r23);
-          const float2 e01 = __ffma2_rn(q01, make_float2(ns.x, ns.y), x01);
-          const float2 e23 = __ffma2_rn(q23, make_float2(ns.z, ns.w), x23);
-          v[q][2 * h] = __ffma2_rn(e01, r01, q01);
-          v[q][2 * h + 1] = __ffma2_rn(e23, r23, q23);
+          v[q][2 * h] = markstein2(x01, r01, make_float2(ns.x, ns.y));
+          v[q][2 * h + 1] = markstein2(x23, r23, make_float2(ns.z, ns.w));
           if (F8) {  // RN(-0 / s) = -0, which Markstein's correction turns into +0; E4M3 keeps the sign
             v[q][2 * h] = make_float2(with_sign_of(v[q][2 * h].x, x01.x), with_sign_of(v[q][2 * h].y, x01.y));
             v[q][2 * h + 1] = make_float2(with_sign_of(v[q][2 * h + 1].x, x23.x), with_sign_of(v[q][2 * h + 1].y, x23.y));

@@ -144,10 +144,8 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
               // Markstein: q = RN(x y), r = x - s q exact, RN(q + r y) = RN(x / s), two lanes at a time
               const float2 x01 = make_float2(d[0], d[1]), x23 = make_float2(d[2], d[3]);
               const float2 r01 = make_float2(rv.x, rv.y), r23 = make_float2(rv.z, rv.w);
-              const float2 q01 = __fmul2_rn(x01, r01), q23 = __fmul2_rn(x23, r23);
-              const float2 e01 = __ffma2_rn(q01, make_float2(-sv.x, -sv.y), x01);
-              const float2 e23 = __ffma2_rn(q23, make_float2(-sv.z, -sv.w), x23);
-              const float2 y01 = __ffma2_rn(e01, r01, q01), y23 = __ffma2_rn(e23, r23, q23);
+              const float2 y01 = markstein2(x01, r01, make_float2(-sv.x, -sv.y));
+              const float2 y23 = markstein2(x23, r23, make_float2(-sv.z, -sv.w));
               d[0] = y01.x; d[1] = y01.y; d[2] = y23.x; d[3] = y23.y;
             } else {
               d[0] = __fdiv_rn(d[0], sv.x);
