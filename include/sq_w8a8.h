@@ -166,8 +166,12 @@ sq_status sq_ln_smooth_quant_per_tensor(const void* x, sq_dtype dt, int64_t M, i
  *   size (16-byte aligned rows take the vectorised store path).  M == 0 or N == 0 is a
  *   no-op; K == 0 is invalid.
  *   workspace: device scratch of at least sq_w8a8_gemm_workspace_size(M, N, K) bytes
- *   (may be NULL when that size is 0), 256-byte aligned; its contents on entry do not
- *   matter.  Calls that share a workspace must be ordered on one stream. */
+ *   (may be NULL when that size is 0), 256-byte aligned.  Zero-fill it once before its first
+ *   use (cudaMemset, torch.zeros): it holds sums of the split work that must start at zero,
+ *   and every call leaves all of it zero-filled again, so one
+ *   workspace serves any number of calls and shapes (and the FP8 GEMM) without clearing.  (A
+ *   call whose kernel stopped on a bounded wait -- sq_device_error() != 0 -- may leave it
+ *   dirty: zero it again.)  Calls that share a workspace must be ordered on one stream. */
 sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                        int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                        void* workspace, size_t ws_bytes, void* stream);
@@ -194,9 +198,10 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *   - The first call on a device looks up the scratch array's device address (set-up, once
  *     per device, with that device current); make that first call before any stream
  *     capture.  A failed look-up returns SQ_ERR_CUDA.
- *   - Every call on a device shares the one array, which keeps the last call's contents;
- *     each call overwrites the partial sums it reads, so nothing needs to start at zero.
- *     Calls that overlap on the GPU (different streams, no ordering) race on it. */
+ *   - Every call on a device shares the one array, which keeps the last call's contents.
+ *     The set-up zero-fills it once (the split-work sums must start at zero, see
+ *     sq_w8a8_gemm); every call leaves it zero-filled again.  Calls that overlap on the GPU
+ *     (different streams, no ordering) race on it. */
 sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                                int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                                void* stream);

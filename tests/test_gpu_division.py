@@ -7,7 +7,7 @@ step.  Markstein's theorem makes that exact as long as no intermediate leaves th
 these tests check it exhaustively where the kernels rely on it:
   * every divisor significand of the binade [1, 2), and of the two binades at the ends of the
     range where the kernels take the fast path (2^-90 and 2^89), against 256 (64 at the ends)
-    dividends whose quotients cover 2^-11 .. 256 -- every magnitude that decides an INT8 or
+    dividends whose quotients cover 2^-12 .. 256 -- every magnitude that decides an INT8 or
     E4M3 code (|v / scale| <= 127 for a scale taken from the data's own absmax);
   * the device's IEEE division itself against the host's (numpy float32 division) on a random
     sample, so the reference of the exhaustive sweeps is pinned to an independent implementation.
@@ -31,7 +31,7 @@ def binade(e: int, sign: float = 1.0) -> torch.Tensor:
 
 def dividends(n: int, e_div: int, seed: int) -> torch.Tensor:
     """n dividends a = +-m 2^(e_div + k), m uniform in [1, 2) with random low bits, k in -11 .. 7, so
-    that a / b for b in [2^e_div, 2^(e_div+1)) lies in 2^-11 .. 256."""
+    that a / b for b in [2^e_div, 2^(e_div+1)) lies in 2^-12 .. 256."""
     rng = np.random.default_rng(seed)
     m = (np.uint32(127 << 23) | rng.integers(0, 1 << 23, n, dtype=np.uint32)).view(np.float32)
     k = rng.integers(-11, 8, n)
@@ -58,7 +58,7 @@ def test_every_divisor_of_a_binade(sign):
 
 @pytest.mark.parametrize("e", [-90, 89])
 def test_binades_at_the_ends_of_the_fast_range(e):
-    a = dividends(64, e, 2 + e)
+    a = dividends(64, e, 200 + e)
     bad_scalar, bad_packed, checked = run(a, binade(e))
     assert checked == 64 << 23
     assert bad_scalar == 0 and bad_packed == 0
@@ -82,7 +82,7 @@ def test_device_reference_matches_host_ieee_division():
     bd, ad = torch.from_numpy(b).to(DEV), torch.from_numpy(a).to(DEV)
     counts, q = sq.sq_selfcheck_shared_divisor(ad, bd, want_quotients=True)
     host = (a[None, :] / b[:, None]).astype(np.float32)  # numpy float32 division: IEEE, nearest even
-    assert np.abs(host).min() >= 2.0 ** -12 and np.abs(host).max() <= 2.0 ** 9
+    assert np.abs(host).min() >= 2.0 ** -12 and np.abs(host).max() <= 2.0 ** 13
     got = q.cpu().numpy()
     # the scalar quotients the library uses equal the host's IEEE quotients bit for bit
     assert np.array_equal(got.view(np.uint32), host.view(np.uint32))

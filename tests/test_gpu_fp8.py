@@ -115,7 +115,7 @@ def _acc_bound(xq, wq):
 
 GEMM_SHAPES = [(1, 8, 16), (1, 200, 272), (7, 24, 32), (16, 256, 256), (16, 4096, 4096), (64, 130, 1024),
                (100, 1000, 512), (129, 264, 128), (256, 512, 4096), (300, 1024, 1040), (2048, 512, 96),
-               (5, 1000, 8192), (7, 5120, 2048)]
+               (5, 1000, 8192), (7, 5120, 2048), (1, 19072, 272), (16, 28672, 1024), (3, 4096, 14336)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -127,6 +127,30 @@ def test_gemm_fp8_accumulator(M, N, K):
     exact, _ = O.fp8_gemm(xq, ones_m, wq, ones_n, "f32")
     err = np.abs(got.astype(np.float64) - exact)
     assert np.all(err <= _acc_bound(xq, wq)), float(np.max(err / np.maximum(_acc_bound(xq, wq), 1e-300)))
+
+
+def test_gemm_fp8_and_int8_share_a_workspace():
+    """FP8 and INT8 GEMMs of split shapes take turns on one zero-filled workspace: every result
+    holds (FP8 within its bound, and the same bits on a repeated call; INT8 exact) and the
+    workspace is all zero after each call."""
+    shapes = [(16, 4096, 4096), (1, 28672, 4096), (300, 1024, 1040), (64, 6144, 4096)]
+    ws = torch.zeros(max(sq.sq_w8a8_gemm_workspace_size(*sh) for sh in shapes), dtype=torch.uint8, device=DEV)
+    rng = np.random.default_rng(21)
+    for M, N, K in shapes:
+        xq, wq = _finite_codes(rng, (M, K)), _finite_codes(rng, (N, K))
+        ones_m, ones_n = np.ones(M, np.float32), np.ones(N, np.float32)
+        a = sq.sq_w8a8_gemm_fp8(dev(xq), dev(ones_m), dev(wq), dev(ones_n), out_dtype=torch.float32, workspace=ws)
+        assert not ws.any()
+        b = sq.sq_w8a8_gemm_fp8(dev(xq), dev(ones_m), dev(wq), dev(ones_n), out_dtype=torch.float32, workspace=ws)
+        assert not ws.any()
+        exact, _ = O.fp8_gemm(xq, ones_m, wq, ones_n, "f32")
+        assert np.all(np.abs(host(a).astype(np.float64) - exact) <= _acc_bound(xq, wq))
+        assert np.array_equal(host(a), host(b))  # a fixed order of additions: reproducible
+        iq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        iw = rng.integers(-127, 128, (N, K)).astype(np.int8)
+        acc = sq.sq_w8a8_gemm(dev(iq), None, dev(iw), None, out_dtype=torch.int32, workspace=ws)
+        assert not ws.any()
+        assert np.array_equal(host(acc), O.w8a8_gemm(iq, None, iw, None, "i32"))
 
 
 @pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (300, 1024, 1040), (2048, 512, 96)])

@@ -308,6 +308,12 @@ GEMM_SHAPES = [
     (100, 1000, 512), (128, 512, 128), (129, 264, 128), (200, 777, 400), (256, 512, 4096),
     (300, 1024, 1040), (1000, 300, 160), (2048, 512, 96),
     (5, 1000, 8192), (7, 5120, 2048),  # decode shapes split 16 and 3 ways
+    # decode shapes whose weight tiles are shared by several CTAs (stream-K): 1.5 tiles per CTA,
+    # 128-token columns, ~5 CTAs per tile over a long K, and two full waves of whole tiles
+    (1, 28672, 4096), (128, 12288, 1024), (16, 4096, 49152), (2, 36864, 256),
+    # whole tiles in a full wave plus one tile split over a few CTAs (most CTAs' split ranges empty),
+    # and two full waves plus a split remainder
+    (1, 19072, 272), (64, 40960, 1024),
 ]
 
 
@@ -337,6 +343,21 @@ def test_gemm_output_leading_dimension():
     sq.sq_w8a8_gemm(dev(xq), dev(sx), dev(wq), dev(sw), y=ybuf[:, :N])
     assert assert_bf16_close(host(ybuf[:, :N].contiguous()), O.w8a8_gemm(xq, sx, wq, sw, "bf16")) == 1.0
     assert (host(ybuf[:, N:].float()) == -1.0).all()
+
+
+def test_gemm_workspace_reused_across_calls_and_shapes():
+    """One zero-filled workspace serves calls of different shapes in turn (stream-K tile sums,
+    split-K partials): all of it is back at zero after every call, and every result is exact."""
+    shapes = [(16, 4096, 4096), (1, 28672, 4096), (64, 6144, 4096), (16, 4096, 4096), (3, 1000, 14336),
+              (256, 512, 4096), (1, 28672, 4096)]
+    need = max(sq.sq_w8a8_gemm_workspace_size(*sh) for sh in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    rng = np.random.default_rng(5)
+    for M, N, K in shapes:
+        xq, wq = random_codes(rng, M, K, extreme_row=0), random_codes(rng, N, K)
+        acc = sq.sq_w8a8_gemm(dev(xq), None, dev(wq), None, out_dtype=torch.int32, workspace=ws)
+        assert np.array_equal(host(acc), O.w8a8_gemm(xq, None, wq, None, "i32"))
+        assert not ws.any()
 
 
 def test_gemm_workspace_too_small_is_reported():

@@ -61,10 +61,13 @@ def inputs(M, N, K, seed):
     return xq, sx, wq, sw
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (64, 6144, 4096), (3, 1000, 14336), (200, 512, 1024)])
+@pytest.mark.parametrize("M,N,K", [(16, 4096, 4096), (64, 6144, 4096), (3, 1000, 14336), (200, 512, 1024),
+                                   (1, 28672, 4096)])
 def test_noalloc_matches_workspace_gemm_on_two_calls(M, N, K):
     need = sq.sq_w8a8_gemm_workspace_size(M, N, K)
-    assert 0 < need <= scratch_bytes()  # these shapes split K, so the scratch is in use
+    if not 0 < need <= scratch_bytes():
+        pytest.skip(f"on this device the launch for {M}x{N}x{K} needs {need} bytes of scratch (premise: 0 < need "
+                    f"<= {scratch_bytes()})")
     xq, sx, wq, sw = inputs(M, N, K, M + N + K)
     ref_y = sq.sq_w8a8_gemm(xq, sx, wq, sw)
     ref_acc = sq.sq_w8a8_gemm(xq, None, wq, None, out_dtype=torch.int32)
@@ -89,8 +92,12 @@ def test_noalloc_without_split_and_after_a_different_shape():
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    M, N, K = 1536, 1536, 4096
-    assert sq.sq_w8a8_gemm_workspace_size(M, N, K) > scratch_bytes()
+    # the first candidate whose launch on this device needs more scratch than the array holds
+    candidates = [(1536, 1536, 4096), (128, 5120, 4096), (2048, 2048, 8192), (4096, 4096, 4096)]
+    big = [c for c in candidates if sq.sq_w8a8_gemm_workspace_size(*c) > scratch_bytes()]
+    if not big:
+        pytest.skip("no candidate shape needs more than the built-in scratch on this device")
+    M, N, K = big[0]
     xq, sx, wq, sw = inputs(M, N, K, 3)
     y = torch.zeros(M, N, dtype=torch.bfloat16, device=DEV)
     assert call_noalloc(xq, sx, wq, sw, y) == 5  # SQ_ERR_WORKSPACE, nothing launched

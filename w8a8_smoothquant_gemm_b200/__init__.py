@@ -279,7 +279,7 @@ def sq_w8a8_gemm(xq: torch.Tensor, sx: torch.Tensor | None, wq: torch.Tensor, sw
         _vec(sw, N, "sw")
     need = sq_w8a8_gemm_workspace_size(M, N, K)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=xq.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)  # its counters start at zero
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("sq_w8a8_gemm", lib().sq_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
                                               y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))
@@ -386,7 +386,7 @@ def sq_w8a8_gemm_fp8(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: t
     _vec(sw, N, "sw")
     need = sq_w8a8_gemm_workspace_size(M, N, K)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=xq.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)  # its counters start at zero
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("sq_w8a8_gemm_fp8", lib().sq_w8a8_gemm_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
                                                       y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))

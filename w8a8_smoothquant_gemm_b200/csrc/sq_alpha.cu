@@ -285,6 +285,8 @@ sq_status sq_alpha_search(const void* x, sq_dtype dt, int64_t M, int64_t K, int6
   const bool ln = gamma != nullptr;
   const AlphaWs w = carve(workspace, M, K, N, ln);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the GEMM's workspace starts zeroed (its tile sums); the caller's buffer may hold anything
+  if (w.gemm_ws) SQ_TRY_CUDA(cudaMemsetAsync(w.gemm_ws, 0, w.gemm_ws_bytes, st));
 
   // statistics of the layer input and the weights (the checks of these calls cover x and W)
   if (ln) SQ_TRY(sq_calib_ln_absmax(x, dt, M, K, ldx, gamma, beta, eps, 0, w.ax, stream));

@@ -22,10 +22,15 @@
 //               next tile's MMAs run meanwhile.
 // Operands are K-major: A = xq [M, K], B = wq [N, K].  For decode-sized M (<= 128) the
 // roles swap (A = wq, B = xq) so the weights fill the 128-row MMA dimension and the
-// tokens the N dimension; when there are fewer tiles than SMs, K is split and int32
-// partials are summed (exactly, in a fixed order) by a second kernel that also applies
-// the epilogue.  Every mbarrier wait is bounded: on expiry the kernel records a code in
-// a device error word and leaves.
+// tokens the N dimension.  When the weight tiles do not fill the SMs evenly, the work is
+// split stream-K style: the tiles' K blocks are laid end to end and every CTA takes an equal
+// run of them, so a tile may be shared by a few CTAs; each adds its int32 partial tile into the
+// tile's sum in the workspace, and a reduction kernel launched behind the GEMM (already
+// resident, waiting on the GEMM grid) applies the epilogue to the shared tiles and puts their
+// sums back to zero.  For M > 128 with fewer tiles than SMs, K is split and the same kind of
+// second kernel sums the partials.
+// Every mbarrier wait is bounded: on expiry the kernel records a code in a device error
+// word and leaves.
 #include <cuda.h>
 
 #include <algorithm>
@@ -57,6 +62,16 @@ struct GemmParams {
   int ydt;                   // SQ_BF16, SQ_F32 or SQ_I32
   int vec_store;             // y and every output row start on a 16-byte boundary
   int32_t* ws;               // [splits][M][N] int32 partials when splits > 1
+  // stream-K (swap layout only): the first sk_dp_tiles tiles go whole to the CTAs in full waves
+  // (tile u to CTA u mod G); of the rest, CTA c of G = sk_ctas takes iterations
+  // [c I / G, (c+1) I / G) of their I = (tiles_a - sk_dp_tiles) * num_kb (tile, K block)
+  // iterations laid end to end
+  int sk;
+  int sk_ctas;
+  int sk_dp_tiles;
+  int64_t sk_iters;
+  int32_t* partials;         // INT8: [tiles_a][BN][BM] int32 tile sums, zero at rest; FP8: [2 * sk_ctas][BN][BM]
+                             // partial tiles, two slots per CTA (both column-major)
 };
 
 // TMA load whose completion is signalled on the mbarrier of the pair's leader CTA
@@ -231,6 +246,63 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta,
   }
 }
 
+// The sequence of pieces (tile, K-block range) one CTA works on.  Data-parallel: units
+// unit0, unit0 + step, ... (decode_unit).  Stream-K: the CTA's iteration range, cut at tile
+// boundaries (the first and last piece may be partial tiles).
+struct Work {
+  int64_t it, end;  // stream-K cursor
+  int u, step;      // data-parallel cursor
+};
+
+__device__ __forceinline__ Work work_begin(const GemmParams& p, int unit0, int unit_step) {
+  Work w;
+  w.u = unit0;
+  w.step = unit_step;
+  w.it = (int64_t)unit0 * p.sk_iters / p.sk_ctas;
+  w.end = (int64_t)(unit0 + 1) * p.sk_iters / p.sk_ctas;
+  return w;
+}
+
+__device__ __forceinline__ bool next_piece(const GemmParams& p, Work& w, int& ta, int& tb, int& kb0, int& kb1,
+                                           int& split) {
+  if (p.sk) {
+    tb = 0;
+    split = 0;
+    if (w.u < p.sk_dp_tiles) {  // whole tiles of the full waves
+      ta = w.u;
+      kb0 = 0;
+      kb1 = p.num_kb;
+      w.u += w.step;
+      return true;
+    }
+    if (w.it >= w.end) return false;
+    const int t_rel = (int)(w.it / p.num_kb);
+    ta = p.sk_dp_tiles + t_rel;
+    kb0 = (int)(w.it - (int64_t)t_rel * p.num_kb);
+    kb1 = (int)min((int64_t)p.num_kb, (int64_t)kb0 + (w.end - w.it));
+    w.it += kb1 - kb0;
+    return true;
+  }
+  if (w.u >= p.num_units) return false;
+  decode_unit(p, w.u, ta, tb, split);
+  kb0 = split * p.kb_per_split;
+  kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+  w.u += w.step;
+  return true;
+}
+
+// Stream-K bookkeeping over the split tiles (t_rel = tile - sk_dp_tiles): the CTA whose
+// iteration range holds split iteration i, and the workspace slot of CTA c's piece of split
+// tile t_rel (slot 2c: the piece in the tile where c's range starts; 2c + 1: where it ends --
+// the only two pieces of a CTA that can be partial).
+__device__ __forceinline__ int sk_owner(const GemmParams& p, int64_t i) {
+  return (int)(((i + 1) * p.sk_ctas + p.sk_iters - 1) / p.sk_iters - 1);
+}
+__device__ __forceinline__ int sk_slot(const GemmParams& p, int c, int t_rel) {
+  const int64_t first = (int64_t)c * p.sk_iters / p.sk_ctas;
+  return 2 * c + ((int)(first / p.num_kb) == t_rel ? 0 : 1);
+}
+
 // Shared-memory layout of one CTA: BN_CTA rows of B per stage (BN / CG), BN accumulator
 // columns per TMEM buffer.
 template <int BN, int STAGES, int CG>
@@ -269,9 +341,6 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::BAR_OFFSET + L::NUM_BARS * 8);
 
-  // a split-K reduction launched behind this grid may be scheduled now (it waits for this
-  // grid's completion before reading anything); without one this is a no-op
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
@@ -309,6 +378,18 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+  // Launched as a programmatic dependent of the previous kernel on the stream: the set-up above
+  // overlaps its tail.  In the swap layout the weights are the streamed operand; the producer
+  // asks L2 for this CTA's first weight tiles before waiting.  A prefetch only fills L2, the
+  // point of coherence, so it is safe even if the previous kernel writes those weights: every
+  // read of the operands, scales and workspace comes after the wait.
+  if (SWAP && warp == 0 && lane == 0) {
+    Work w = work_begin(p, unit0, unit_step);
+    int ta, tb, kb0, kb1, split, n = 0;
+    while (n < STAGES && next_piece(p, w, ta, tb, kb0, kb1, split))
+      for (int kb = kb0; kb < kb1 && n < STAGES; ++kb, ++n) tma_prefetch_l2(&map_a, kb * BK, ta * BM);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (each CTA)
@@ -318,11 +399,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       bool ok = true;
       uint32_t issued = 0;  // bit s: stage s has been loaded; its last load used parity bit s of `par`
       uint32_t par = 0;
-      for (int u = unit0; u < p.num_units && ok; u += unit_step) {
-        int ta, tb, split;
-        decode_unit(p, u, ta, tb, split);
-        const int kb0 = split * p.kb_per_split;
-        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      Work w = work_begin(p, unit0, unit_step);
+      int ta, tb, kb0, kb1, split;
+      while (ok && next_piece(p, w, ta, tb, kb0, kb1, split)) {
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
             atomicOr(&g_error_word, ERR_GEMM_PRODUCER_WAIT);
@@ -348,6 +427,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           }
         }
       }
+      // every load of this CTA is issued: the kernel launched behind this grid (the split
+      // reduction, or the next GEMM) may be scheduled now; it waits for this grid's completion
+      // before it reads anything
+      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
       if (!ok && leader) {
         // let the loads issued for this barrier land before the block exits (bounded, 100 ms)
         for (int s = 0; s < STAGES; ++s)
@@ -361,11 +444,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int u = unit0; u < p.num_units && ok; u += unit_step, ++it) {
-        int ta, tb, split;
-        decode_unit(p, u, ta, tb, split);
-        const int kb0 = split * p.kb_per_split;
-        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      Work w = work_begin(p, unit0, unit_step);
+      int ta, tb, kb0, kb1, split;
+      for (; ok && next_piece(p, w, ta, tb, kb0, kb1, split); ++it) {
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(tempty_bar(acc), aph ^ 1u)) {
@@ -404,9 +485,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;          // row of this CTA's A tile = TMEM lane
     int it = 0;
-    for (int u = unit0; u < p.num_units; u += unit_step, ++it) {
-      int ta, tb, split;
-      decode_unit(p, u, ta, tb, split);
+    Work w = work_begin(p, unit0, unit_step);
+    int ta, tb, kb0, kb1, split;
+    for (; next_piece(p, w, ta, tb, kb0, kb1, split); ++it) {
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       if (!mbar_wait(tfull_bar(acc), aph)) {
@@ -418,6 +499,28 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int64_t arow = (int64_t)ta * MMA_M + (int64_t)rank * BM + row;
       constexpr int CH = BN >= 32 ? 32 : 16;
+      if (SWAP && p.sk && !(kb0 == 0 && kb1 == p.num_kb)) {
+        // ---- a partial tile (stream-K): INT8 adds it into the tile's int32 sum (exact in any
+        // order), FP8 writes it to this CTA's slot; the reduction kernel that follows this grid
+        // finishes the tile
+        const int t_rel = ta - p.sk_dp_tiles;
+        int32_t* dst = p.partials + (int64_t)(F8 ? sk_slot(p, (int)blockIdx.x, t_rel) : t_rel) * (BM * BN) + row;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += CH) {
+          uint32_t r[CH];
+          tmem_ld<CH>(taddr + (uint32_t)c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            if (F8) __stcg(dst + (c0 + i) * BM, (int)r[i]);
+            else atomicAdd(dst + (c0 + i) * BM, (int)r[i]);  // return value unused: a reduction
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += CH) {
         uint32_t r[CH];
@@ -469,18 +572,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           // A row = output column n; TMEM columns = output rows m
           const int64_t n = arow;
           const int64_t m0 = (int64_t)tb * BN + c0;
-          if (n < p.N) {
-            if (p.splits > 1) {
-              for (int i = 0; i < CH; ++i) {
-                const int64_t m = m0 + i;
-                if (m < p.M) p.ws[((int64_t)split * p.M + m) * p.N + n] = (int32_t)r[i];
-              }
-            } else {
-              const float swn = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n);
-              for (int i = 0; i < CH; ++i) {
-                const int64_t m = m0 + i;
-                if (m < p.M) store_out<F8>(p, m, n, r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
-              }
+          if (n < p.N) {  // (swap-layout tiles are whole here: partial ones took the stream-K branch)
+            const float swn = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n);
+            for (int i = 0; i < CH; ++i) {
+              const int64_t m = m0 + i;
+              if (m < p.M) store_out<F8>(p, m, n, r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
             }
           }
         }
@@ -512,11 +608,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 }
 
 
-// Sums the split-K partials in split order (int32: exact; F8: fp32 in that fixed order) and
-// applies the epilogue.
+// Sums the split-K partials in split order (int32: exact; F8: fp32 in that fixed order),
+// applies the epilogue and zeroes the partials (the workspace is zero at rest).
 template <bool F8>
 __global__ void __launch_bounds__(256)
-splitk_reduce_kernel(const int32_t* __restrict__ ws, int splits, int64_t M, int64_t N, const float* __restrict__ sx,
+splitk_reduce_kernel(int32_t* __restrict__ ws, int splits, int64_t M, int64_t N, const float* __restrict__ sx,
                      const float* __restrict__ sw, void* __restrict__ y, int64_t ldy, int ydt) {
   // launched as a programmatic dependent of the GEMM: its blocks may be resident before the
   // GEMM ends, and wait here until the GEMM grid has completed and its partials are visible
@@ -533,6 +629,7 @@ splitk_reduce_kernel(const int32_t* __restrict__ ws, int splits, int64_t M, int6
       for (int s = 0; s < splits; ++s) a += ws[(int64_t)s * total + i];
       acc = (uint32_t)a;
     }
+    for (int s = 0; s < splits; ++s) ws[(int64_t)s * total + i] = 0;
     const int64_t m = i / N, n = i % N;
     const int64_t off = m * ldy + n;
     if (ydt == SQ_BF16)
@@ -541,6 +638,54 @@ splitk_reduce_kernel(const int32_t* __restrict__ ws, int splits, int64_t M, int6
       reinterpret_cast<float*>(y)[off] = dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n));
     else
       reinterpret_cast<int32_t*>(y)[off] = (int32_t)acc;
+  }
+}
+
+// Finishes the tiles of a stream-K GEMM that several CTAs shared: y = epilogue(sum of the
+// partial tiles), and the workspace back to zero.  INT8: the int32 tile sum; FP8: the
+// contributors' slots added in K order.  Block b covers 1024 elements of split tile b / (BN / 8)
+// (column-major inside the tile): each thread four consecutive rows n of one column m.
+template <bool F8>
+__global__ void __launch_bounds__(256)
+sk_reduce_kernel(const GemmParams p, int bn) {
+  // the next kernel on the stream may start its set-up now; this grid's work waits for the GEMM
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int chunks = bn / 8;  // BM * bn / 1024
+  const int t_rel = (int)(blockIdx.x / chunks);
+  const int c_first = sk_owner(p, (int64_t)t_rel * p.num_kb);
+  const int c_last = sk_owner(p, (int64_t)(t_rel + 1) * p.num_kb - 1);
+  if (c_first == c_last) return;  // a whole tile: the GEMM stored it
+  const int per_tile = BM * bn;
+  const int e = (int)(blockIdx.x % chunks) * 1024 + threadIdx.x * 4;  // element of the tile
+  const int col = e / BM, row = e % BM;
+  uint32_t acc[4];
+  if (!F8) {
+    int4* a = reinterpret_cast<int4*>(p.partials + (int64_t)t_rel * per_tile + e);
+    const int4 v = __ldcg(a);
+    __stcg(a, make_int4(0, 0, 0, 0));
+    acc[0] = (uint32_t)v.x; acc[1] = (uint32_t)v.y; acc[2] = (uint32_t)v.z; acc[3] = (uint32_t)v.w;
+  } else {
+    float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int c = c_first; c <= c_last; ++c) {
+      int4* a = reinterpret_cast<int4*>(p.partials + (int64_t)sk_slot(p, c, t_rel) * per_tile + e);
+      const int4 v = __ldcg(a);
+      __stcg(a, make_int4(0, 0, 0, 0));
+      sum[0] = __fadd_rn(sum[0], __int_as_float(v.x));
+      sum[1] = __fadd_rn(sum[1], __int_as_float(v.y));
+      sum[2] = __fadd_rn(sum[2], __int_as_float(v.z));
+      sum[3] = __fadd_rn(sum[3], __int_as_float(v.w));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = __float_as_uint(sum[i]);
+  }
+  const int64_t m = col;
+  if (m >= p.M) return;
+  const float sxm = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t n = (int64_t)(p.sk_dp_tiles + t_rel) * BM + row + i;
+    if (n < p.N) store_out<F8>(p, m, n, acc[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n));
   }
 }
 
@@ -591,7 +736,10 @@ struct GemmPlan {
   int cg;  // CTAs per MMA tile (2: a CTA pair computes 256-row tiles)
   int bn;
   int tiles_a, tiles_b, num_kb, kb_per_split, splits;
-  size_t ws_bytes;
+  bool sk;          // stream-K split of the swap layout
+  int sk_ctas, sk_dp_tiles;
+  int64_t sk_iters;
+  size_t ws_bytes;  // 0, or the split-K partials / stream-K tile sums (zero at rest)
 };
 
 static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
@@ -599,18 +747,36 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
   const int sms = num_sms();
   pl.swap = M <= 128;
   pl.cg = 1;
+  pl.num_kb = (int)((K + sqk::BK - 1) / sqk::BK);
   if (pl.swap) {
     pl.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
     pl.tiles_a = (int)((N + sqk::BM - 1) / sqk::BM);
     pl.tiles_b = 1;
-  } else {
-    pl.bn = 256;
-    pl.cg = 2;
-    const int64_t tile_m = (int64_t)sqk::BM * pl.cg;
-    pl.tiles_a = (int)((M + tile_m - 1) / tile_m);
-    pl.tiles_b = (int)((N + pl.bn - 1) / pl.bn);
+    pl.splits = 1;
+    pl.kb_per_split = pl.num_kb;
+    // Weight streaming: every SM should stream the same number of bytes.  Whole tiles per CTA
+    // when they fill the SMs within 10%; otherwise stream-K, at least 4 K blocks (64 KB of
+    // weights) per CTA.
+    const int64_t tiles = pl.tiles_a;
+    const int64_t waves = (tiles + sms - 1) / sms;
+    if (tiles * 10 < waves * sms * 9) {
+      // whole tiles in the full waves, stream-K over the remaining tiles
+      pl.sk = true;
+      pl.sk_dp_tiles = (int)(tiles / sms * sms);
+      const int64_t split_tiles = tiles - pl.sk_dp_tiles;
+      pl.sk_iters = split_tiles * pl.num_kb;
+      pl.sk_ctas = pl.sk_dp_tiles ? sms : (int)std::min<int64_t>(sms, std::max<int64_t>(1, pl.sk_iters / 4));
+      // int32 tile sums (INT8) or two partial slots per CTA (FP8), whichever is larger
+      const int64_t tiles_or_slots = std::max<int64_t>(split_tiles, 2 * (int64_t)pl.sk_ctas);
+      pl.ws_bytes = (size_t)tiles_or_slots * sqk::BM * pl.bn * sizeof(int32_t);
+    }
+    return pl;
   }
-  pl.num_kb = (int)((K + sqk::BK - 1) / sqk::BK);
+  pl.bn = 256;
+  pl.cg = 2;
+  const int64_t tile_m = (int64_t)sqk::BM * pl.cg;
+  pl.tiles_a = (int)((M + tile_m - 1) / tile_m);
+  pl.tiles_b = (int)((N + pl.bn - 1) / pl.bn);
   const int64_t tiles = (int64_t)pl.tiles_a * pl.tiles_b;
   const int slots = sms / pl.cg;  // tiles that run at once
   int splits = 1;
@@ -634,23 +800,22 @@ static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, cons
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
   if (e != cudaSuccess) return e;
   const int slots = num_sms() / CG;
-  const int grid = std::min(p.num_units, slots) * CG;
-  if (CG == 1) {
-    kern<<<grid, sqk::GEMM_THREADS, L::TOTAL, st>>>(ma, mb, p);
-    return cudaGetLastError();
-  }
+  const int grid = p.sk ? p.sk_ctas : std::min(p.num_units, slots) * CG;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(sqk::GEMM_THREADS);
   cfg.dynamicSmemBytes = L::TOTAL;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  // programmatic dependent launch: the CTAs' set-up may overlap the previous kernel's tail
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CG;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = CG == 1 ? 1 : 2;
   return cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
 }
 
@@ -700,7 +865,13 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   p.ydt = ydt;
   const int64_t elt = ydt == SQ_BF16 ? 2 : 4;
   p.vec_store = (reinterpret_cast<uintptr_t>(y) % 16 == 0) && (ldy * elt) % 16 == 0;
-  p.ws = static_cast<int32_t*>(ws);
+  // workspace (zero at rest): split-K partials, or the stream-K tile sums / slots
+  p.ws = pl.ws_bytes ? static_cast<int32_t*>(ws) : nullptr;
+  p.partials = p.ws;
+  p.sk = pl.sk ? 1 : 0;
+  p.sk_ctas = pl.sk ? pl.sk_ctas : 1;
+  p.sk_dp_tiles = pl.sk ? pl.sk_dp_tiles : 0;
+  p.sk_iters = pl.sk ? pl.sk_iters : 1;
   cudaError_t e;
   if (!pl.swap) {
     e = launch_cfg<256, 6, false, 2, F8>(ma, mb, p, st);
@@ -712,7 +883,22 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
       default: e = launch_cfg<128, 6, true, 1, F8>(ma, mb, p, st); break;
     }
   }
-  if (e != cudaSuccess || pl.splits == 1) return e;
+  if (e != cudaSuccess) return e;
+  if (pl.sk) {
+    // the shared tiles' reduction, a programmatic dependent of the GEMM (resident while it runs)
+    const int64_t blocks = (int64_t)(pl.tiles_a - pl.sk_dp_tiles) * (pl.bn / 8);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, sqk::sk_reduce_kernel<F8>, p, pl.bn);
+  }
+  if (pl.splits == 1) return e;
   const int64_t total = M * N;
   const int64_t grid = std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 16);
   // programmatic dependent launch: the reduction's launch overlaps the GEMM's tail
@@ -725,8 +911,7 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sqk::splitk_reduce_kernel<F8>, static_cast<const int32_t*>(ws), pl.splits, M, N,
-                            sx, sw, y, ldy, ydt);
+  return cudaLaunchKernelEx(&cfg, sqk::splitk_reduce_kernel<F8>, p.ws, pl.splits, M, N, sx, sw, y, ldy, ydt);
 }
 
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,

@@ -39,7 +39,12 @@ cudaError_t scratch_address(void** addr) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(g_scratch_once[dev], [dev] {
     void* p = nullptr;
-    g_scratch_status[dev] = cudaGetSymbolAddress(&p, g_gemm_scratch);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_gemm_scratch);
+    // the GEMM's split-work sums in the scratch must start at zero; every call leaves them at zero
+    // again (a synchronous memset: this set-up precedes any stream capture)
+    if (e == cudaSuccess) e = cudaMemset(p, 0, SQ_NOALLOC_SCRATCH_BYTES);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    g_scratch_status[dev] = e;
     g_scratch_addr[dev] = p;
   });
   if (g_scratch_status[dev] != cudaSuccess) return g_scratch_status[dev];
