@@ -412,6 +412,31 @@ def quantizer_profile(sq, layers, reps=3) -> dict:
     return out
 
 
+def next_linear_fused(sq, up, down, hbm_gbs) -> dict:
+    """The down linear's quantiser fused into the up linear's GEMM: the up GEMM (with the down
+    linear's smoothing folded into its output scales) stores the down input and its row maxima,
+    and a codes pass quantises it; against the same GEMM followed by the full per-token quantiser
+    (statistics pass + codes pass over the stored output)."""
+    M, N = up.M, up.N
+    sw2 = sq.sq_fold_next_smoothing(up.sw, down.s)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=up.x.device)
+    rmax = torch.empty(M, dtype=torch.float32, device=up.x.device)
+    xq = torch.empty(M, N, dtype=torch.int8, device=up.x.device)
+    sx = torch.empty(M, dtype=torch.float32, device=up.x.device)
+    ones = torch.ones(N, dtype=torch.float32, device=up.x.device)
+    t_gemm = time_graph(lambda: sq.sq_w8a8_gemm(up.xq, up.sx, up.wq, sw2, y=y, workspace=up.ws), 4)
+    t_gemm_rm = time_graph(lambda: sq.sq_w8a8_gemm_rowmax(up.xq, up.sx, up.wq, sw2, y=y, rowmax=rmax,
+                                                          workspace=up.ws), 4)
+    t_quant = time_graph(lambda: sq.sq_ln_smooth_quant(y, s=ones, xq=xq, sx=sx), 8)
+    t_codes = time_graph(lambda: sq.sq_quant_codes(y, rmax, xq=xq, sx=sx), 8)
+    b_codes = M * N * 3 + 8 * M
+    return {"workload": f"up {M}x{N}x{up.K} GEMM -> down input {M}x{N}",
+            "gemm_us": round(t_gemm * 1e6, 1), "gemm_rowmax_us": round(t_gemm_rm * 1e6, 1),
+            "quantiser_us": round(t_quant * 1e6, 1), "codes_pass_us": round(t_codes * 1e6, 1),
+            "codes_pass_hbm_frac": round(b_codes / t_codes / 1e9 / hbm_gbs, 3),
+            "unfused_us": round((t_gemm + t_quant) * 1e6, 1), "fused_us": round((t_gemm_rm + t_codes) * 1e6, 1)}
+
+
 def calibration_config(sq, device, hbm_gbs) -> dict:
     """The calibration reduction: per-channel absmax over 512 x 512 tokens x 4096 bf16 channels
     (2 GiB, ~1% channels x log-uniform [20, 100]), the weight absmax of W [4096, 4096] and s for
@@ -690,6 +715,7 @@ def run_device(args, rank, world, local):
                                      "median over the timed steps"}
     launches = count_launches(sq, layers, world)
     decode_175 = {} if args.quick else decode_sweep(sq, layers, DECODE_M_175B, hbm)
+    next2 = next_linear_fused(sq, layers[2], layers[3], hbm)
     quant_175 = quantizer_profile(sq, layers)
     e2e = e2e_measure(sq, layers, world, device, max(2, args.steps // 10), ops_step)
 
@@ -734,6 +760,7 @@ def run_device(args, rank, world, local):
                              "step (L2 126 MB)",
                        "parallelism": f"dp{world}"},
             "roofline": roofline, "headline": headline, "quantizer": quant_175, "decode_175b": decode_175,
+            "next_linear_fused": next2,
             "prefill_8b": prefill8, "decode_8b": decode_8b, "calibration": calib,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": None if launches is None else launches * args.steps,

@@ -176,6 +176,31 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, cons
                        int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* sq_w8a8_gemm_rowmax -- sq_w8a8_gemm whose epilogue also emits the per-row max of the output,
+ * for a linear whose output is the next linear's input ("4.2 W8A8 量化与 SmoothQuant", sec. 6:
+ * the input of a linear comes from a LayerNorm or from the previous GEMM's output, and the
+ * smoothing folds into that previous layer; "量化：只压权重，与训练后量化（PTQ）", SmoothQuant section).
+ * With the next linear's factors folded into sw (sq_fold_next_smoothing), y is already the next
+ * linear's smoothed input, and
+ *   rowmax[m] = max_n |y[m, n]|  over the values as stored (bf16-rounded for SQ_BF16),
+ * which is exactly the statistic the next per-token quantiser would compute by reading y;
+ * sq_quant_codes then finishes the quantisation in one read of y.
+ *   Arguments as for sq_w8a8_gemm except: ydt is SQ_BF16 or SQ_F32; rowmax: fp32 [M] device
+ *   array, 4-byte aligned, overwritten (the call zero-fills it before the GEMM runs). */
+sq_status sq_w8a8_gemm_rowmax(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                              int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
+                              float* rowmax, void* workspace, size_t ws_bytes, void* stream);
+
+/* sq_quant_codes -- the codes pass of the per-token quantiser for rows whose max is known
+ * (from sq_w8a8_gemm_rowmax): sx[m] = rowmax[m] / 127 (binary32, correctly rounded);
+ * xq[m, j] = clamp(rne(x[m, j] / sx[m]), -127, 127) (a zero max gives zero codes).  With rowmax
+ * the row maxima of x this equals sq_ln_smooth_quant(x, plain mode, s = 1) bit for bit, with
+ * one read of x ("SmoothQuant大模型平滑量化技术", Python demo: max/127, round, clip).
+ *   x: [M, K] bf16/fp32, ldx (16-byte aligned rows); rowmax: fp32 [M]; xq: int8 [M, K] dense,
+ *   16-byte aligned; sx: fp32 [M].  K % 16 == 0 (no upper limit: rows are not held on chip). */
+sq_status sq_quant_codes(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx, const float* rowmax,
+                         int8_t* xq, float* sx, void* stream);
+
 /* Workspace bytes sq_w8a8_gemm needs for this shape on the current device (0 when the
  * launch it picks does not split K).  Returns (size_t)-1 for invalid sizes. */
 size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);

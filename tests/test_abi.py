@@ -165,6 +165,27 @@ def test_gemm_noalloc_checks_arguments_before_its_scratch_size():
     assert call(M=0) == 0
 
 
+def test_gemm_rowmax_and_codes_validation():
+    g = sq.lib().sq_w8a8_gemm_rowmax
+
+    def call(xq=A16, sx=A16b, wq=A16c, sw=A16b, M=8, N=32, K=64, y=A16, ydt=BF16, ldy=32, rmax=A16b, ws=NULL, wsb=0):
+        return g(xq, sx, wq, sw, M, N, K, y, ydt, ldy, rmax, ws, wsb, NULL)
+
+    assert call(ydt=I32) == INVALID          # the row max needs scaled outputs
+    assert call(rmax=NULL) == INVALID
+    assert call(rmax=ctypes.c_void_p(0x10002)) == INVALID
+    assert call(xq=NULL) == INVALID
+    assert call(K=40) == ALIGN
+    assert call(M=0) == 0
+    c = sq.lib().sq_quant_codes
+    assert c(A16, BF16, 4, 64, 64, NULL, A16b, A16c, NULL) == INVALID       # null rowmax
+    assert c(A16, BF16, 4, 0, 0, A16b, A16b, A16c, NULL) == INVALID         # K = 0
+    assert c(A16, BF16, 4, 24, 24, A16b, A16b, A16c, NULL) == ALIGN         # 48-byte rows
+    assert c(A16, BF16, 4, 64, 64, A16b, A8, A16c, NULL) == ALIGN           # misaligned codes
+    assert c(A16, I32, 4, 64, 64, A16b, A16b, A16c, NULL) == INVALID        # int32 input
+    assert c(A16, BF16, 0, 64, 64, NULL, NULL, NULL, NULL) == 0             # nothing to do
+
+
 def test_workspace_size_validation():
     f = sq.lib().sq_w8a8_gemm_workspace_size
     assert f(4, 4, 0) == ctypes.c_size_t(-1).value

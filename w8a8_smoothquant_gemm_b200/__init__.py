@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
             "sq_fold_kernel_launches": [P, I, I64, I64, I64],
             "sq_alpha_search": [P, I, I64, I64, I64, P, P, F, P, I, I64, I64, P, I, P, P, SZ, P],
             "sq_selfcheck_shared_divisor": [P, I64, P, I64, P, P, P],
+            "sq_w8a8_gemm_rowmax": [P, P, P, P, I64, I64, I64, P, I, I64, P, P, SZ, P],
+            "sq_quant_codes": [P, I, I64, I64, I64, P, P, P, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -284,6 +286,49 @@ def sq_w8a8_gemm(xq: torch.Tensor, sx: torch.Tensor | None, wq: torch.Tensor, sw
     _check("sq_w8a8_gemm", lib().sq_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), ydt,
                                               y.stride(0), _ptr(workspace), ws_bytes, _stream(stream)))
     return y
+
+
+def sq_w8a8_gemm_rowmax(xq: torch.Tensor, sx: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                        out_dtype: torch.dtype = torch.bfloat16, y: torch.Tensor | None = None,
+                        rowmax: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """sq_w8a8_gemm that also returns rowmax[m] = max_n |y[m, n]| of the stored outputs (the next
+    linear's per-token statistic).  Returns (y, rowmax)."""
+    if xq.dtype != torch.int8 or wq.dtype != torch.int8 or not xq.is_contiguous() or not wq.is_contiguous():
+        raise ValueError("xq and wq must be contiguous int8 tensors")
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError("xq and wq disagree on K")
+    if y is None:
+        y = torch.empty(M, N, dtype=out_dtype, device=xq.device)
+    if rowmax is None:
+        rowmax = torch.empty(M, dtype=torch.float32, device=xq.device)
+    _vec(sx, M, "sx")
+    _vec(sw, N, "sw")
+    _vec(rowmax, M, "rowmax")
+    need = sq_w8a8_gemm_workspace_size(M, N, K)
+    if workspace is None and need > 0:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=xq.device)  # its sums start at zero
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("sq_w8a8_gemm_rowmax", lib().sq_w8a8_gemm_rowmax(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y),
+                                                            _ODT[y.dtype], y.stride(0), _ptr(rowmax), _ptr(workspace),
+                                                            ws_bytes, _stream(stream)))
+    return y, rowmax
+
+
+def sq_quant_codes(x: torch.Tensor, rowmax: torch.Tensor, xq: torch.Tensor | None = None,
+                   sx: torch.Tensor | None = None, stream=None):
+    """Per-token INT8 codes of x given its row maxima: (xq [M, K] int8, sx [M] = rowmax / 127)."""
+    x = _mat(x, "x")
+    M, K = x.shape
+    _vec(rowmax, M, "rowmax")
+    if xq is None:
+        xq = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check("sq_quant_codes", lib().sq_quant_codes(_ptr(x), _dt(x), M, K, x.stride(0), _ptr(rowmax), _ptr(xq), _ptr(sx),
+                                                  _stream(stream)))
+    return xq, sx
 
 
 # ----------------------------------------------------------------------------- alpha search

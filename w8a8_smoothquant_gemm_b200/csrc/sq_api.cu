@@ -24,8 +24,10 @@ cudaError_t launch_ln_smooth_quant_per_tensor(const void* x, bool bf16, int64_t 
                                               int static_scale, float* scale, int8_t* xq, float* sx,
                                               cudaStream_t st);
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
-                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
-                        bool* ws_too_small);
+                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, float* rowmax,
+                        cudaStream_t st, bool* ws_too_small);
+cudaError_t launch_quant_codes(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* rowmax,
+                               int8_t* xq, float* sx, cudaStream_t st);
 cudaError_t launch_fold_next_smoothing(const float* sw, const float* s_next, int64_t N, float* out, cudaStream_t st);
 cudaError_t launch_fold_quant_fp8(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw, const float* s,
                                   const float* gamma, const float* beta, uint8_t* Wq, float* sw, float* gamma_f,
@@ -307,10 +309,38 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, cons
   const sq_status st = check_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, workspace, true, &empty);
   if (st != SQ_OK || empty) return st;
   bool ws_small = false;
-  cudaError_t err = sqh::launch_gemm(xq, sx, wq, sw, M, N, K, y, (int)ydt, ldy, workspace, ws_bytes,
+  cudaError_t err = sqh::launch_gemm(xq, sx, wq, sw, M, N, K, y, (int)ydt, ldy, workspace, ws_bytes, nullptr,
                                      as_stream(stream), &ws_small);
   if (ws_small) return SQ_ERR_WORKSPACE;
   return cuda_status(err);
+}
+
+sq_status sq_w8a8_gemm_rowmax(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M,
+                              int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy, float* rowmax, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  if (ydt != SQ_BF16 && ydt != SQ_F32) return SQ_ERR_INVALID_ARG;
+  bool empty = false;
+  const sq_status st = check_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, workspace, false, &empty);
+  if (st != SQ_OK || empty) return st;
+  if (rowmax == nullptr || !aligned4(rowmax)) return SQ_ERR_INVALID_ARG;
+  bool ws_small = false;
+  cudaError_t err = sqh::launch_gemm(xq, sx, wq, sw, M, N, K, y, (int)ydt, ldy, workspace, ws_bytes, rowmax,
+                                     as_stream(stream), &ws_small);
+  if (ws_small) return SQ_ERR_WORKSPACE;
+  return cuda_status(err);
+}
+
+sq_status sq_quant_codes(const void* x, sq_dtype dt, int64_t M, int64_t K, int64_t ldx, const float* rowmax, int8_t* xq,
+                         float* sx, void* stream) {
+  if (M < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_matrix(x, dt, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if (M == 0) return SQ_OK;
+  if (rowmax == nullptr || !aligned4(rowmax) || xq == nullptr || sx == nullptr || !aligned4(sx))
+    return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || !aligned16(xq)) return SQ_ERR_ALIGNMENT;
+  if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
+  return cuda_status(sqh::launch_quant_codes(x, dt == SQ_BF16, M, K, ldx, rowmax, xq, sx, as_stream(stream)));
 }
 
 sq_status sq_device_error(unsigned int* code, int clear, void* stream) {

@@ -23,6 +23,13 @@ enum : unsigned int {
   ERR_ROW_TMA_WAIT = 1u << 4,
 };
 
+// max(a, b, c) in one instruction (three-operand max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // bf16 bits -> fp32 (exact widening).
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

@@ -72,6 +72,7 @@ struct GemmParams {
   int64_t sk_iters;
   int32_t* partials;         // INT8: [tiles_a][BN][BM] int32 tile sums, zero at rest; FP8: [2 * sk_ctas][BN][BM]
                              // partial tiles, two slots per CTA (both column-major)
+  float* rowmax;             // NULL, or [M]: running max over n of |y[m, n]| as stored (zeroed before the launch)
 };
 
 // TMA load whose completion is signalled on the mbarrier of the pair's leader CTA
@@ -211,13 +212,31 @@ __device__ __forceinline__ float dequant(uint32_t acc, float sxm, float swn) {
   return __fmul_rn(__fmul_rn(acc_value<F8>(acc), sxm), swn);
 }
 
+// Stores one output and returns its magnitude as stored (the bf16 value for bf16 output; 0 for
+// raw int32 output, which has no row max).
 template <bool F8>
-__device__ __forceinline__ void store_out(const GemmParams& p, int64_t m, int64_t n, uint32_t acc, float sxm,
-                                          float swn) {
+__device__ __forceinline__ float store_out(const GemmParams& p, int64_t m, int64_t n, uint32_t acc, float sxm,
+                                           float swn) {
   const int64_t off = m * p.ldy + n;
-  if (p.ydt == SQ_BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(dequant<F8>(acc, sxm, swn));
-  else if (p.ydt == SQ_F32) reinterpret_cast<float*>(p.y)[off] = dequant<F8>(acc, sxm, swn);
-  else reinterpret_cast<int32_t*>(p.y)[off] = (int32_t)acc;
+  if (p.ydt == SQ_BF16) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(dequant<F8>(acc, sxm, swn));
+    reinterpret_cast<__nv_bfloat16*>(p.y)[off] = h;
+    return fabsf(__bfloat162float(h));
+  }
+  if (p.ydt == SQ_F32) {
+    const float v = dequant<F8>(acc, sxm, swn);
+    reinterpret_cast<float*>(p.y)[off] = v;
+    return fabsf(v);
+  }
+  reinterpret_cast<int32_t*>(p.y)[off] = (int32_t)acc;
+  return 0.0f;
+}
+
+// Max over the 32 lanes of a warp (every lane gets it).
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
 // Unit u -> (A tile, B tile, K split).  Splits of one tile are adjacent so they run
@@ -379,11 +398,12 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
   // Launched as a programmatic dependent of the previous kernel on the stream: the set-up above
-  // overlaps its tail.  In the swap layout the weights are the streamed operand; the producer
-  // asks L2 for this CTA's first weight tiles before waiting.  A prefetch only fills L2, the
-  // point of coherence, so it is safe even if the previous kernel writes those weights: every
-  // read of the operands, scales and workspace comes after the wait.
-  if (SWAP && warp == 0 && lane == 0) {
+  // overlaps its tail.  In the swap layout the weights are the streamed operand; an epilogue
+  // warp (idle until the first accumulator) asks L2 for this CTA's first weight tiles before
+  // waiting.  A prefetch only fills L2, the point of coherence, so it is safe even if the
+  // previous kernel writes those weights: every read of the operands, scales and workspace
+  // comes after the wait.
+  if (SWAP && warp == 2 && lane == 0) {
     Work w = work_begin(p, unit0, unit_step);
     int ta, tb, kb0, kb1, split, n = 0;
     while (n < STAGES && next_piece(p, w, ta, tb, kb0, kb1, split))
@@ -499,6 +519,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int64_t arow = (int64_t)ta * MMA_M + (int64_t)rank * BM + row;
       constexpr int CH = BN >= 32 ? 32 : 16;
+      float rmax = 0.0f;  // this thread's output row: max |y| over the tile's columns (rowmax mode)
       if (SWAP && p.sk && !(kb0 == 0 && kb1 == p.num_kb)) {
         // ---- a partial tile (stream-K): INT8 adds it into the tile's int32 sum (exact in any
         // order), FP8 writes it to this CTA's slot; the reduction kernel that follows this grid
@@ -546,6 +567,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                   const float v1 = dequant<F8>(r[i + 1], sxm, __ldg(p.sw + n0 + i + 1));
                   __nv_bfloat162 h = __halves2bfloat162(__float2bfloat16_rn(v0), __float2bfloat16_rn(v1));
                   packed[i / 2] = *reinterpret_cast<uint32_t*>(&h);
+                  rmax = fmax3(rmax, fabsf(__low2float(h)), fabsf(__high2float(h)));
                 }
                 uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y) + m * p.ldy + n0);
 #pragma unroll
@@ -556,14 +578,16 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
                 for (int v = 0; v < CH / 4; ++v) {  // (sw is only 4-byte aligned: scalar loads)
                   const float* w = p.sw + n0 + 4 * v;
-                  dst[v] = make_float4(dequant<F8>(r[4 * v], sxm, __ldg(w)), dequant<F8>(r[4 * v + 1], sxm, __ldg(w + 1)),
-                                       dequant<F8>(r[4 * v + 2], sxm, __ldg(w + 2)),
-                                       dequant<F8>(r[4 * v + 3], sxm, __ldg(w + 3)));
+                  const float4 o = make_float4(dequant<F8>(r[4 * v], sxm, __ldg(w)), dequant<F8>(r[4 * v + 1], sxm, __ldg(w + 1)),
+                                               dequant<F8>(r[4 * v + 2], sxm, __ldg(w + 2)),
+                                               dequant<F8>(r[4 * v + 3], sxm, __ldg(w + 3)));
+                  dst[v] = o;
+                  rmax = fmax3(rmax, fmax3(fabsf(o.x), fabsf(o.y), fabsf(o.z)), fabsf(o.w));
                 }
               } else {
                 for (int i = 0; i < CH; ++i) {
                   const int64_t n = n0 + i;
-                  if (n < p.N) store_out<F8>(p, m, n, r[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n));
+                  if (n < p.N) rmax = fmaxf(rmax, store_out<F8>(p, m, n, r[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n)));
                 }
               }
             }
@@ -572,15 +596,20 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           // A row = output column n; TMEM columns = output rows m
           const int64_t n = arow;
           const int64_t m0 = (int64_t)tb * BN + c0;
-          if (n < p.N) {  // (swap-layout tiles are whole here: partial ones took the stream-K branch)
-            const float swn = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n);
-            for (int i = 0; i < CH; ++i) {
-              const int64_t m = m0 + i;
-              if (m < p.M) store_out<F8>(p, m, n, r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
+          // (swap-layout tiles are whole here: partial ones took the stream-K branch)
+          const float swn = (p.ydt == SQ_I32 || n >= p.N) ? 0.0f : __ldg(p.sw + n);
+          for (int i = 0; i < CH; ++i) {
+            const int64_t m = m0 + i;
+            float a = 0.0f;
+            if (m < p.M && n < p.N) a = store_out<F8>(p, m, n, r[i], p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m), swn);
+            if (p.rowmax) {  // output row m spans the lanes (one output column n per lane)
+              a = warp_max(a);
+              if (lane == 0 && m < p.M) atomic_max_nonneg(p.rowmax + m, a);
             }
           }
         }
       }
+      if (!SWAP && p.rowmax && p.splits == 1 && arow < p.M) atomic_max_nonneg(p.rowmax + arow, rmax);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -613,7 +642,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 template <bool F8>
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(int32_t* __restrict__ ws, int splits, int64_t M, int64_t N, const float* __restrict__ sx,
-                     const float* __restrict__ sw, void* __restrict__ y, int64_t ldy, int ydt) {
+                     const float* __restrict__ sw, void* __restrict__ y, int64_t ldy, int ydt, float* rowmax) {
   // launched as a programmatic dependent of the GEMM: its blocks may be resident before the
   // GEMM ends, and wait here until the GEMM grid has completed and its partials are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -632,12 +661,17 @@ splitk_reduce_kernel(int32_t* __restrict__ ws, int splits, int64_t M, int64_t N,
     for (int s = 0; s < splits; ++s) ws[(int64_t)s * total + i] = 0;
     const int64_t m = i / N, n = i % N;
     const int64_t off = m * ldy + n;
-    if (ydt == SQ_BF16)
-      reinterpret_cast<__nv_bfloat16*>(y)[off] = __float2bfloat16_rn(dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n)));
-    else if (ydt == SQ_F32)
-      reinterpret_cast<float*>(y)[off] = dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n));
-    else
+    if (ydt == SQ_BF16) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n)));
+      reinterpret_cast<__nv_bfloat16*>(y)[off] = h;
+      if (rowmax) atomic_max_nonneg(rowmax + m, fabsf(__bfloat162float(h)));
+    } else if (ydt == SQ_F32) {
+      const float v = dequant<F8>(acc, __ldg(sx + m), __ldg(sw + n));
+      reinterpret_cast<float*>(y)[off] = v;
+      if (rowmax) atomic_max_nonneg(rowmax + m, fabsf(v));
+    } else {
       reinterpret_cast<int32_t*>(y)[off] = (int32_t)acc;
+    }
   }
 }
 
@@ -679,13 +713,18 @@ sk_reduce_kernel(const GemmParams p, int bn) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = __float_as_uint(sum[i]);
   }
-  const int64_t m = col;
+  const int64_t m = col;  // the same for the 32 lanes of a warp (32 x 4 rows = one column of the tile)
   if (m >= p.M) return;
   const float sxm = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m);
+  float a = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t n = (int64_t)(p.sk_dp_tiles + t_rel) * BM + row + i;
-    if (n < p.N) store_out<F8>(p, m, n, acc[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n));
+    if (n < p.N) a = fmaxf(a, store_out<F8>(p, m, n, acc[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n)));
+  }
+  if (p.rowmax) {
+    a = warp_max(a);
+    if ((threadIdx.x & 31) == 0) atomic_max_nonneg(p.rowmax + m, a);
   }
 }
 
@@ -822,10 +861,14 @@ static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, cons
 template <bool F8>
 static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* wq, const float* sw, int64_t M,
                                    int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
-                                   cudaStream_t st, bool* ws_too_small) {
+                                   float* rowmax, cudaStream_t st, bool* ws_too_small) {
   const GemmPlan pl = plan_gemm(M, N, K);
   *ws_too_small = pl.ws_bytes > 0 && (ws == nullptr || ws_bytes < pl.ws_bytes);
   if (*ws_too_small) return cudaSuccess;
+  if (rowmax) {  // the epilogue takes a running max into it
+    const cudaError_t ez = cudaMemsetAsync(rowmax, 0, sizeof(float) * (size_t)M, st);
+    if (ez != cudaSuccess) return ez;
+  }
   CUtensorMap ma, mb;
   const void* a_ptr = pl.swap ? (const void*)wq : (const void*)xq;
   const void* b_ptr = pl.swap ? (const void*)xq : (const void*)wq;
@@ -872,6 +915,7 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   p.sk_ctas = pl.sk ? pl.sk_ctas : 1;
   p.sk_dp_tiles = pl.sk ? pl.sk_dp_tiles : 0;
   p.sk_iters = pl.sk ? pl.sk_iters : 1;
+  p.rowmax = rowmax;
   cudaError_t e;
   if (!pl.swap) {
     e = launch_cfg<256, 6, false, 2, F8>(ma, mb, p, st);
@@ -911,20 +955,20 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sqk::splitk_reduce_kernel<F8>, p.ws, pl.splits, M, N, sx, sw, y, ldy, ydt);
+  return cudaLaunchKernelEx(&cfg, sqk::splitk_reduce_kernel<F8>, p.ws, pl.splits, M, N, sx, sw, y, ldy, ydt, rowmax);
 }
 
 cudaError_t launch_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M, int64_t N,
-                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, cudaStream_t st,
-                        bool* ws_too_small) {
-  return launch_gemm_any<false>(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, ws_bytes, st, ws_too_small);
+                        int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes, float* rowmax,
+                        cudaStream_t st, bool* ws_too_small) {
+  return launch_gemm_any<false>(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, ws_bytes, rowmax, st, ws_too_small);
 }
 
 // FP8 variant: E4M3 codes, fp32 accumulation, the same epilogue (ydt BF16 or F32).
 cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw, int64_t M,
                             int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
                             cudaStream_t st, bool* ws_too_small) {
-  return launch_gemm_any<true>(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, ws_bytes, st, ws_too_small);
+  return launch_gemm_any<true>(xq, sx, wq, sw, M, N, K, y, ydt, ldy, ws, ws_bytes, nullptr, st, ws_too_small);
 }
 
 // Device address of the error word on the current device (for kernels in other files).

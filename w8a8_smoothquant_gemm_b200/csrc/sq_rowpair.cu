@@ -38,13 +38,6 @@ namespace sqk {
 
 enum PairMode : int { PAIR_LN_QUANT = 0, PAIR_PLAIN_QUANT = 1, PAIR_LN_CALIB = 2 };
 
-// max(a, b, c) in one instruction (three-operand max.f32, sm_100).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
 // Lane that holds the total of group i after the transposed butterfly over P groups (the
 // exchange at distance 16 >> k decides bit (log2 P - 1 - k) of the group index).
 template <int P>
