@@ -299,7 +299,10 @@ sq_status sq_w8a8_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq
                            void* workspace, size_t ws_bytes, void* stream);
 
 /* Reads (and with clear != 0 resets) the device-side error word of the current device:
- * 0 when no kernel gave up on a bounded wait.  Synchronises `stream`. */
+ * 0 when no kernel gave up on a bounded wait.  Synchronises `stream`.  Bits: 1, 2, 4 -- a GEMM
+ * wait (producer, tensor-core issue, epilogue); 8 -- a weight-fold copy; 16 -- an activation-row
+ * copy.  A kernel whose wait runs out stops at once: it lets the copies it has already issued
+ * land (each within 100 ms), takes no further work and leaves; its outputs are then undefined. */
 sq_status sq_device_error(unsigned int* code, int clear, void* stream);
 
 /* sq_selfcheck_shared_divisor -- checks, on the device, the division every quantiser and the
@@ -317,6 +320,13 @@ sq_status sq_device_error(unsigned int* code, int clear, void* stream);
  *   uint64, 8-byte aligned, accumulated into (zero them first).  All device pointers. */
 sq_status sq_selfcheck_shared_divisor(const float* a, int64_t na, const float* b, int64_t nb, float* q,
                                       unsigned long long* counts, void* stream);
+
+/* sq_set_wait_limit -- the limit of every bounded wait in this library's kernels on the
+ * current device (default 10 s; the setting outlasts the call, for this process only).  A
+ * diagnostic: 0 makes every wait run out at once, so that a test can drive each kernel's
+ * give-up path (error bit, drain, early exit) without a GPU fault.  Synchronises `stream`.
+ * The pages have no counterpart. */
+sq_status sq_set_wait_limit(unsigned long long ns, void* stream);
 
 /* Human-readable name of a status. */
 const char* sq_status_string(sq_status status);

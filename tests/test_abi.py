@@ -186,6 +186,11 @@ def test_gemm_rowmax_and_codes_validation():
     assert c(A16, BF16, 0, 64, 64, NULL, NULL, NULL, NULL) == 0             # nothing to do
 
 
+def test_wait_limit_symbol():
+    f = sq.lib().sq_set_wait_limit
+    assert f.argtypes[0] is ctypes.c_uint64
+
+
 def test_workspace_size_validation():
     f = sq.lib().sq_w8a8_gemm_workspace_size
     assert f(4, 4, 0) == ctypes.c_size_t(-1).value

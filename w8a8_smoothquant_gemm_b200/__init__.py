@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "sq_selfcheck_shared_divisor": [P, I64, P, I64, P, P, P],
             "sq_w8a8_gemm_rowmax": [P, P, P, P, I64, I64, I64, P, I, I64, P, P, SZ, P],
             "sq_quant_codes": [P, I, I64, I64, I64, P, P, P, P],
+            "sq_set_wait_limit": [ctypes.c_uint64, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -449,6 +450,14 @@ def sq_selfcheck_shared_divisor(a: torch.Tensor, b: torch.Tensor, want_quotients
     _check("sq_selfcheck_shared_divisor", lib().sq_selfcheck_shared_divisor(_ptr(a), a.numel(), _ptr(b), b.numel(),
                                                                             _ptr(q), _ptr(counts), _stream(stream)))
     return counts, q
+
+
+WAIT_LIMIT_DEFAULT_NS = 10 * 1000 * 1000 * 1000
+
+
+def sq_set_wait_limit(ns: int, stream=None) -> None:
+    """Limit of the kernels' bounded waits on this device (0: every wait runs out at once)."""
+    _check("sq_set_wait_limit", lib().sq_set_wait_limit(int(ns), _stream(stream)))
 
 
 def sq_device_error(clear: bool = True, stream=None) -> int:

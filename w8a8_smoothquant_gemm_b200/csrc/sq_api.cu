@@ -41,6 +41,7 @@ cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* w
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 int fold_kernel_launches(const void* W, bool bf16, int64_t K, int64_t N, int64_t ldw);
 cudaError_t read_device_error(unsigned int* code, int clear, cudaStream_t st);
+cudaError_t set_wait_limit(unsigned long long ns, cudaStream_t st);
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -341,6 +342,10 @@ sq_status sq_quant_codes(const void* x, sq_dtype dt, int64_t M, int64_t K, int64
   if (K % 16 != 0 || !aligned16(xq)) return SQ_ERR_ALIGNMENT;
   if (M > (int64_t)INT32_MAX) return SQ_ERR_UNSUPPORTED;
   return cuda_status(sqh::launch_quant_codes(x, dt == SQ_BF16, M, K, ldx, rowmax, xq, sx, as_stream(stream)));
+}
+
+sq_status sq_set_wait_limit(unsigned long long ns, void* stream) {
+  return cuda_status(sqh::set_wait_limit(ns, as_stream(stream)));
 }
 
 sq_status sq_device_error(unsigned int* code, int clear, void* stream) {

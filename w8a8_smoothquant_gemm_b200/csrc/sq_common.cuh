@@ -13,8 +13,23 @@
 
 namespace sqk {
 
-// Codes OR-ed into the device-side error word (defined next to the GEMM, the only
-// kernel with waits) when a bounded wait runs out; read with sq_device_error().
+// Device-side diagnostics (one per device, defined next to the GEMM): the error word that a
+// kernel whose bounded wait ran out ORs its code into (read with sq_device_error()), and the
+// limit of those waits (sq_set_wait_limit(); 0 makes every wait run out at once).  Kernels in
+// other files get the address of `error` and read the limit beside it.
+struct DeviceDiag {
+  unsigned int error;
+  unsigned int reserved;
+  unsigned long long wait_limit_ns;
+};
+
+__device__ __forceinline__ unsigned long long wait_limit(const unsigned int* err) {
+  return reinterpret_cast<const volatile DeviceDiag*>(err)->wait_limit_ns;
+}
+
+// Limit of the waits that let copies already issued land before a kernel that gave up leaves.
+constexpr unsigned long long DRAIN_NS = 100ull * 1000 * 1000;
+
 enum : unsigned int {
   ERR_GEMM_PRODUCER_WAIT = 1u << 0,
   ERR_GEMM_MMA_WAIT = 1u << 1,

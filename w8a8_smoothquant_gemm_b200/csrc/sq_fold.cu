@@ -319,6 +319,7 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
 
   const int tid = threadIdx.x;
   const uint32_t crank = cluster_ctarank();
+  const unsigned long long limit = wait_limit(err);
   const int64_t strip = blockIdx.x / C;
   const int64_t k0 = strip * CW;
   const int64_t j0 = (int64_t)crank * RK;
@@ -348,13 +349,17 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
 
   // ---- partial column max of |s_j W_jk| over this CTA's rows, piece by piece as they land:
   // thread = 8 columns x rows rl, rl + G, ...
+  bool failed = false;
   {
     const int cg = tid % (CW / 8), rl = tid / (CW / 8);
     float m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = 0.0f;
     for (int p = 0; p < pieces; ++p) {
-      if (!mbar_wait(smem_u32(&bars[p]), 0)) atomicOr(err, ERR_FOLD_TMA_WAIT);
+      if (!mbar_wait(smem_u32(&bars[p]), 0, limit)) {
+        failed = true;  // stop reading this block; the cluster exchange below still takes place
+        break;
+      }
       for (int j = p * 64 + rl; j < p * 64 + 64; j += G) {
         const uint4 w = *reinterpret_cast<const uint4*>(tile + j * CW + cg * 8);
         const float2 sj = make_float2(s_rows[j], s_rows[j]);
@@ -371,7 +376,11 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[rl][cg * 8 + e] = m[e];
   }
-  __syncthreads();
+  failed = __syncthreads_or(failed);
+  if (failed && tid == 0) {
+    atomicOr(err, ERR_FOLD_TMA_WAIT);
+    for (int p = 0; p < pieces; ++p) (void)mbar_wait(smem_u32(&bars[p]), 0, DRAIN_NS);  // issued copies land
+  }
   if (tid < CW) {
     float m = red[0][tid];
     for (int g = 1; g < G; ++g) m = fmaxf(m, red[g][tid]);
@@ -387,8 +396,8 @@ fold_cluster_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, int64_t
   }
   __syncthreads();
 
-  // ---- codes, transposed
-  fold_write_codes<CW, F8>(tile, s_rows, scale, K, N, RK, j0, k0, Wq);
+  // ---- codes, transposed (not after a wait ran out: the block's data is incomplete)
+  if (!failed) fold_write_codes<CW, F8>(tile, s_rows, scale, K, N, RK, j0, k0, Wq);
 }
 
 // ---------------------------------------------------------------------------- two-pass fold
@@ -477,6 +486,7 @@ fold_codes_stream_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, in
   __shared__ float scale[FCS_CW];
   __shared__ __align__(8) uint64_t bars[S];
   const int tid = threadIdx.x;
+  const unsigned long long limit = wait_limit(err);
   const int64_t strips = (N + FCS_CW - 1) / FCS_CW, rtiles = (K + RT - 1) / RT;
   const int64_t units = strips * rtiles;
   const int64_t first = blockIdx.x, step = gridDim.x;
@@ -506,7 +516,17 @@ fold_codes_stream_kernel(const __grid_constant__ CUtensorMap wmap, int64_t K, in
     if (tid < FCS_CW) scale[tid] = (k0 + tid < N) ? __fdiv_rn(__ldg(colmax + k0 + tid), F8 ? 448.0f : 127.0f) : 0.0f;
     __syncthreads();
     const int stage = (int)(i % S);
-    if (!mbar_wait(smem_u32(&bars[stage]), (uint32_t)((i / S) & 1))) atomicOr(err, ERR_FOLD_TMA_WAIT);
+    const bool ok = mbar_wait(smem_u32(&bars[stage]), (uint32_t)((i / S) & 1), limit);
+    if (__syncthreads_or(!ok)) {
+      // the block stops: the tiles it has issued (i .. i + S - 1) land before it leaves
+      if (tid == 0) {
+        atomicOr(err, ERR_FOLD_TMA_WAIT);
+        for (int j = 0; j < S; ++j)
+          if (first + (i + j) * step < units)
+            (void)mbar_wait(smem_u32(&bars[(int)((i + j) % S)]), (uint32_t)(((i + j) / S) & 1), DRAIN_NS);
+      }
+      break;
+    }
     fold_write_codes<FCS_CW, F8, RT>(reinterpret_cast<const uint16_t*>(ring + (size_t)stage * TILE), s_rows, scale,
                                      K, N, RT, j0, k0, Wq);
     __syncthreads();

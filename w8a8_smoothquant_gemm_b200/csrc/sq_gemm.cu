@@ -34,12 +34,13 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstddef>
 
 #include "sq_ptx.cuh"
 
 namespace sqk {
 
-__device__ unsigned int g_error_word = 0;
+__device__ DeviceDiag g_diag = {0u, 0u, WAIT_NS};
 
 constexpr int BM = 128;          // MMA M: rows of the A operand per tile
 constexpr int BK = 128;          // K bytes per ring stage (one 128-byte swizzle row)
@@ -397,6 +398,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+  const unsigned long long limit = g_diag.wait_limit_ns;
   // Launched as a programmatic dependent of the previous kernel on the stream: the set-up above
   // overlaps its tail.  In the swap layout the weights are the streamed operand; an epilogue
   // warp (idle until the first accumulator) asks L2 for this CTA's first weight tiles before
@@ -423,8 +425,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       int ta, tb, kb0, kb1, split;
       while (ok && next_piece(p, w, ta, tb, kb0, kb1, split)) {
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
-            atomicOr(&g_error_word, ERR_GEMM_PRODUCER_WAIT);
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, limit)) {
+            atomicOr(&g_diag.error, ERR_GEMM_PRODUCER_WAIT);
             ok = false;
             break;
           }
@@ -454,7 +456,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       if (!ok && leader) {
         // let the loads issued for this barrier land before the block exits (bounded, 100 ms)
         for (int s = 0; s < STAGES; ++s)
-          if (issued & (1u << s)) (void)mbar_wait(full_bar(s), (par >> s) & 1u, 100ull * 1000 * 1000);
+          if (issued & (1u << s)) (void)mbar_wait(full_bar(s), (par >> s) & 1u, DRAIN_NS);
       }
     }
   } else if (warp == 1) {
@@ -469,15 +471,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       for (; ok && next_piece(p, w, ta, tb, kb0, kb1, split); ++it) {
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-        if (!mbar_wait(tempty_bar(acc), aph ^ 1u)) {
-          atomicOr(&g_error_word, ERR_GEMM_MMA_WAIT);
+        if (!mbar_wait(tempty_bar(acc), aph ^ 1u, limit)) {
+          atomicOr(&g_diag.error, ERR_GEMM_MMA_WAIT);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase)) {
-            atomicOr(&g_error_word, ERR_GEMM_MMA_WAIT);
+          if (!mbar_wait(full_bar(stage), phase, limit)) {
+            atomicOr(&g_diag.error, ERR_GEMM_MMA_WAIT);
             ok = false;
             break;
           }
@@ -510,8 +512,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     for (; next_piece(p, w, ta, tb, kb0, kb1, split); ++it) {
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-      if (!mbar_wait(tfull_bar(acc), aph)) {
-        atomicOr(&g_error_word, ERR_GEMM_EPILOGUE_WAIT);
+      if (!mbar_wait(tfull_bar(acc), aph, limit)) {
+        atomicOr(&g_diag.error, ERR_GEMM_EPILOGUE_WAIT);
         break;
       }
       __syncwarp();  // tcgen05.ld below is .sync.aligned: reconverge after the wait loop
@@ -978,19 +980,25 @@ unsigned int* error_word_ptr() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   if (!ptrs[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, sqk::g_error_word) == cudaSuccess) ptrs[dev] = static_cast<unsigned int*>(p);
+    if (cudaGetSymbolAddress(&p, sqk::g_diag) == cudaSuccess) ptrs[dev] = static_cast<unsigned int*>(p);
   }
   return ptrs[dev];
 }
 
 cudaError_t read_device_error(unsigned int* code, int clear, cudaStream_t st) {
-  cudaError_t e = cudaMemcpyFromSymbolAsync(code, sqk::g_error_word, sizeof(unsigned int), 0,
-                                            cudaMemcpyDeviceToHost, st);
+  cudaError_t e = cudaMemcpyFromSymbolAsync(code, sqk::g_diag, sizeof(unsigned int), 0, cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return e;
   e = cudaStreamSynchronize(st);
   if (e != cudaSuccess || !clear) return e;
   const unsigned int zero = 0;
-  e = cudaMemcpyToSymbolAsync(sqk::g_error_word, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+  e = cudaMemcpyToSymbolAsync(sqk::g_diag, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);
+}
+
+cudaError_t set_wait_limit(unsigned long long ns, cudaStream_t st) {
+  cudaError_t e = cudaMemcpyToSymbolAsync(sqk::g_diag, &ns, sizeof(ns), offsetof(sqk::DeviceDiag, wait_limit_ns),
+                                          cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return e;
   return cudaStreamSynchronize(st);
 }

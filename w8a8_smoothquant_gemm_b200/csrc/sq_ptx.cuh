@@ -44,9 +44,11 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// Waits for the phase with the given parity to complete; false after `limit_ns`.
+// Waits for the phase with the given parity to complete; false after `limit_ns` (a limit of 0
+// runs out at once, without looking at the barrier: the library's test of its error paths).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           unsigned long long limit_ns = WAIT_NS) {
+  if (limit_ns == 0) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {

@@ -37,9 +37,12 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
   uint8_t* ring = reinterpret_cast<uint8_t*>(sb + K);  // [G][S][row_bytes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)G * S * row_bytes);  // [G][S]
   __shared__ float red[G][24];
+  __shared__ int stop[G];  // a group's wait ran out: it takes no further rows
 
   const int gid = threadIdx.x / T, t = threadIdx.x % T;
   const int nchunks = K / 8;
+  const unsigned long long limit = wait_limit(err);
+  if (t == 0) stop[gid] = 0;
 
   // per-channel vectors, once per block, as float4s ordered [half][chunk] (element j sits at
   // ((j % 8) / 4 * nchunks + j / 8) * 4 + j % 4) so that a thread's read of its chunk's half
@@ -86,9 +89,20 @@ rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, c
   for (int64_t r = r0; r < M; r += rstep, ++it) {
     const int slot = (int)(it % S);
     // one lane polls the slot's barrier; the rest of the group sleeps in the group barrier
-    if (t == 0 && !mbar_wait(smem_u32(&bars[gid * S + slot]), (uint32_t)((it / S) & 1)))
+    if (t == 0 && !mbar_wait(smem_u32(&bars[gid * S + slot]), (uint32_t)((it / S) & 1), limit)) {
       atomicOr(err, ERR_ROW_TMA_WAIT);
+      stop[gid] = 1;
+    }
     group_barrier<T>(gid);
+    if (stop[gid]) {
+      // the group stops: the copies it has issued (rows it .. it + S - 1) land before it leaves
+      if (t == 0)
+        for (int j = 0; j < S; ++j)
+          if (r + j * rstep < M)
+            (void)mbar_wait(smem_u32(&bars[gid * S + (int)((it + j) % S)]), (uint32_t)(((it + j) / S) & 1), DRAIN_NS);
+      group_barrier<T>(gid);
+      break;
+    }
     const uint8_t* rowp = gring + (size_t)slot * row_bytes;
     float v[NCH * 8];
 #pragma unroll
