@@ -115,7 +115,8 @@ def _acc_bound(xq, wq):
 
 GEMM_SHAPES = [(1, 8, 16), (1, 200, 272), (7, 24, 32), (16, 256, 256), (16, 4096, 4096), (64, 130, 1024),
                (100, 1000, 512), (129, 264, 128), (256, 512, 4096), (300, 1024, 1040), (2048, 512, 96),
-               (5, 1000, 8192), (7, 5120, 2048), (1, 19072, 272), (16, 28672, 1024), (3, 4096, 14336)]
+               (5, 1000, 8192), (7, 5120, 2048), (1, 19072, 272), (16, 28672, 1024), (3, 4096, 14336),
+               (2048, 12200, 128)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)

@@ -314,6 +314,8 @@ GEMM_SHAPES = [
     # whole tiles in a full wave plus one tile split over a few CTAs (most CTAs' split ranges empty),
     # and two full waves plus a split remainder
     (1, 19072, 272), (64, 40960, 1024),
+    # CTA-pair tiles over several waves, one with a ragged last column tile
+    (2048, 12288, 256), (2048, 12200, 128),
 ]
 
 
