@@ -205,7 +205,8 @@ def test_ln_smooth_quant(dt, M, K, mode):
     assert np.array_equal(host(xq), r_xq)
 
 
-@pytest.mark.parametrize("rows,K", [(1, 256), (100, 4096), (1000, 4096), (70, 8192), (5, 14336), (33, 49152)])
+@pytest.mark.parametrize("rows,K", [(1, 256), (100, 4096), (1000, 4096), (70, 8192), (5, 14336), (33, 49152),
+                                    (20, 12288), (9, 10240), (300, 24576)])
 def test_calib_ln_absmax(rows, K):
     c = sq_inputs.make_case(rows, K, 8, rows + K, beta_std=0.1)
     got = sq.sq_calib_ln_absmax(dev(c.x), dev(c.gamma), dev(c.beta))

@@ -8,6 +8,7 @@
 // per-thread running max, a block reduction, and one atomicMax per column per block on
 // the float bit pattern (monotone for non-negative floats, so the result is exact and
 // independent of order).
+#include "sq_ptx.cuh"
 #include "sq_rowln.cuh"
 
 namespace sqk {
@@ -165,6 +166,10 @@ absmax_rows_warp_kernel(const char* __restrict__ x, int64_t rows, int64_t nvec, 
 // chunks -- in registers (REG, rows of up to 32 elements per thread) or in shared memory --
 // then one atomicMax per column per block.  With rows_atomic set (K too large for shared
 // memory) the running max goes straight to global memory with an atomic per element per row.
+// Launched in clusters (shared-memory maxima only), the blocks of a cluster first combine
+// their maxima through distributed shared memory and each column takes one atomicMax per
+// cluster: with a few rows per block (2048 rows of 12288 on 592 blocks), one atomic per
+// column per block took longer than reading the rows.
 template <bool BF16, int MAXC, bool PREFETCH, bool REG>
 __global__ void __launch_bounds__(ROW_THREADS)
 calib_ln_absmax_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t ld_bytes,
@@ -217,26 +222,54 @@ calib_ln_absmax_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t 
       }
     }
   } else if (!rows_atomic) {
-    __syncthreads();
-    for (int j = threadIdx.x; j < K; j += ROW_THREADS) atomic_max_nonneg(out + j, colmax[j]);
+    const uint32_t C = cluster_nctarank();
+    if (C == 1) {
+      __syncthreads();
+      for (int j = threadIdx.x; j < K; j += ROW_THREADS) atomic_max_nonneg(out + j, colmax[j]);
+    } else {
+      cluster_sync();  // every block's maxima are complete (every block of the cluster gets here)
+      const uint32_t q = cluster_ctarank();
+      const int share = (K + (int)C - 1) / (int)C;
+      const int j1 = min(K, (int)(q + 1) * share);
+      for (int j = (int)q * share + threadIdx.x; j < j1; j += ROW_THREADS) {
+        float m = colmax[j];
+        for (uint32_t p = 0; p < C; ++p)
+          if (p != q) m = fmaxf(m, ld_dsmem_f32(&colmax[j], p));
+        atomic_max_nonneg(out + j, m);
+      }
+      cluster_sync();  // no block leaves while a peer still reads its shared memory
+    }
   }
 }
 
 // Rows of up to 8192 elements: one group of T threads per row (see sq_rowln.cuh), the
 // running column max of the thread's own chunks in registers across all rows the group
 // visits, one atomicMax per column per group at the end.
-template <bool BF16, int T, int NCH>
+// SMEM (T = 256, one row per block; rows of 12288 or 14336 over few tokens): the running
+// maxima live in shared memory instead (48 or 56 KB), which leaves the registers for the
+// prefetched next row at two blocks per SM; launched in clusters, the blocks of a cluster
+// combine their maxima through distributed shared memory, and each column takes one atomicMax
+// per cluster (one per block per column took longer than reading the rows).
+constexpr int CALIB_CLUSTER = 8;
+
+template <bool BF16, int T, int NCH, bool SMEM = false>
 __global__ void __launch_bounds__(256)
 calib_ln_group_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t ld_bytes,
                       const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                       float* __restrict__ out) {
+  static_assert(!SMEM || T == 256, "one row per block with the maxima in shared memory");
   constexpr int G = 256 / T;
   __shared__ float red[G][16];
+  extern __shared__ float colsm[];  // SMEM: [K]
   const int gid = threadIdx.x / T, t = threadIdx.x % T;
   const int nchunks = K / 8;
-  float cm[NCH * 8];
+  float cm[SMEM ? 1 : NCH * 8];
+  if constexpr (SMEM) {
+    for (int j = threadIdx.x; j < K; j += 256) colsm[j] = 0.0f;
+  } else {
 #pragma unroll
-  for (int i = 0; i < NCH * 8; ++i) cm[i] = 0.0f;
+    for (int i = 0; i < NCH * 8; ++i) cm[i] = 0.0f;
+  }
   RowRaw<BF16, NCH> raw;
   const int64_t rstep = (int64_t)gridDim.x * G;
   const int64_t r0 = (int64_t)blockIdx.x * G + gid;
@@ -253,12 +286,51 @@ calib_ln_group_kernel(const char* __restrict__ x, int64_t rows, int K, int64_t l
       if (c < nchunks) {
         float y[8];
         ln_chunk(v + i * 8, mu, rstd, gamma, beta, c, y);
+        if constexpr (SMEM) {
+          float4* d = reinterpret_cast<float4*>(colsm + c * 8);  // this thread's own columns
+          float4 a = d[0], b = d[1];
+          a.x = fmaxf(a.x, fabsf(y[0])); a.y = fmaxf(a.y, fabsf(y[1]));
+          a.z = fmaxf(a.z, fabsf(y[2])); a.w = fmaxf(a.w, fabsf(y[3]));
+          b.x = fmaxf(b.x, fabsf(y[4])); b.y = fmaxf(b.y, fabsf(y[5]));
+          b.z = fmaxf(b.z, fabsf(y[6])); b.w = fmaxf(b.w, fabsf(y[7]));
+          d[0] = a;
+          d[1] = b;
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) cm[i * 8 + e] = fmaxf(cm[i * 8 + e], fabsf(y[e]));
+          for (int e = 0; e < 8; ++e) cm[i * 8 + e] = fmaxf(cm[i * 8 + e], fabsf(y[e]));
+        }
       }
     }
   }
-  if (r0 < rows) {
+  if constexpr (SMEM) {
+    const uint32_t C = cluster_nctarank();
+    if (C == 1) {
+      __syncthreads();
+      if (r0 < rows)
+        for (int j = threadIdx.x; j < K; j += 256) atomic_max_nonneg(out + j, colsm[j]);
+    } else {
+      // clusters of CALIB_CLUSTER blocks; K % (4 * CALIB_CLUSTER) == 0 on this route
+      cluster_sync();  // every block's maxima are complete (every block of the cluster gets here)
+      const uint32_t q = cluster_ctarank();
+      const int share = K / CALIB_CLUSTER;
+      for (int j = (int)q * share + 4 * threadIdx.x; j < (int)(q + 1) * share; j += 4 * 256) {
+        float4 v[CALIB_CLUSTER];  // every CTA's four maxima, all loads in flight at once
+#pragma unroll
+        for (int p = 0; p < CALIB_CLUSTER; ++p) v[p] = ld_dsmem_f32x4(&colsm[j], (uint32_t)p);
+        float4 m = v[0];
+#pragma unroll
+        for (int p = 1; p < CALIB_CLUSTER; ++p) {
+          m.x = fmaxf(m.x, v[p].x); m.y = fmaxf(m.y, v[p].y);
+          m.z = fmaxf(m.z, v[p].z); m.w = fmaxf(m.w, v[p].w);
+        }
+        atomic_max_nonneg(out + j, m.x);
+        atomic_max_nonneg(out + j + 1, m.y);
+        atomic_max_nonneg(out + j + 2, m.z);
+        atomic_max_nonneg(out + j + 3, m.w);
+      }
+      cluster_sync();  // no block leaves while a peer still reads its shared memory
+    }
+  } else if (r0 < rows) {
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = t + T * i;
@@ -331,9 +403,29 @@ static cudaError_t launch_calib_ln_t(const void* x, int64_t rows, int K, int64_t
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sqk::ROW_THREADS, smem);
   if (e != cudaSuccess) return e;
   int64_t grid = std::min<int64_t>(rows, (int64_t)num_sms() * std::max(per_sm, 1));
-  kern<<<(unsigned)grid, sqk::ROW_THREADS, smem, st>>>((const char*)x, rows, K, ld_bytes, gamma, beta, eps,
-                                                       rows_atomic ? 1 : 0, out);
-  return cudaGetLastError();
+  constexpr int CL = 8;  // blocks per cluster when the maxima are in shared memory
+  if (REG || rows_atomic || grid < CL) {
+    kern<<<(unsigned)grid, sqk::ROW_THREADS, smem, st>>>((const char*)x, rows, K, ld_bytes, gamma, beta, eps,
+                                                         rows_atomic ? 1 : 0, out);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(sqk::ROW_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)(grid / CL * CL));
+  int clusters = 0;
+  e = max_active_clusters(reinterpret_cast<const void*>(kern), &cfg, &clusters);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3((unsigned)(CL * std::max<int64_t>(1, std::min<int64_t>(grid / CL, clusters))));
+  return cudaLaunchKernelEx(&cfg, kern, (const char*)x, rows, K, ld_bytes, gamma, beta, eps, 0, out);
 }
 
 int pick_row_threads(int64_t K, int max_nch, int* nch);
@@ -358,6 +450,43 @@ static cudaError_t launch_calib_group_t(const void* x, int64_t rows, int K, int6
   return cudaGetLastError();
 }
 
+// LayerNorm calibration of bf16 rows of 12288 or 14336 (6 or 7 chunks per thread) over few
+// tokens: one row per block, maxima in shared memory, clusters of 8 blocks.
+template <int NCH>
+static cudaError_t launch_calib_smem_t(const void* x, int64_t rows, int K, int64_t ld_bytes, const float* gamma,
+                                       const float* beta, float eps, float* out, cudaStream_t st) {
+  auto kern = sqk::calib_ln_group_kernel<true, 256, NCH, true>;
+  const size_t smem = sizeof(float) * (size_t)K;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 1;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)num_sms() * std::max(per_sm, 1));
+  constexpr int CL = sqk::CALIB_CLUSTER;
+  if (grid < CL) {
+    kern<<<(unsigned)grid, 256, smem, st>>>((const char*)x, rows, K, ld_bytes, gamma, beta, eps, out);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)(grid / CL * CL));
+  int clusters = 0;
+  e = max_active_clusters(reinterpret_cast<const void*>(kern), &cfg, &clusters);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3((unsigned)(CL * std::max<int64_t>(1, std::min<int64_t>(grid / CL, clusters))));
+  return cudaLaunchKernelEx(&cfg, kern, (const char*)x, rows, K, ld_bytes, gamma, beta, eps, out);
+}
+
 template <bool BF16, int T>
 static cudaError_t launch_calib_group_nch(int nch, const void* x, int64_t rows, int K, int64_t ld_bytes,
                                           const float* gamma, const float* beta, float eps, float* out,
@@ -377,6 +506,10 @@ cudaError_t launch_calib_ln_absmax(const void* x, bool bf16, int64_t rows, int64
   const int64_t ldb = ld * (bf16 ? 2 : 4);
   if (rowpair_supported(K, bf16, true, rows))  // chunk-pair rows of the model widths
     return launch_rowpair_calib(x, rows, K, ld, gamma, beta, eps, out, st);
+  if (bf16 && (K == 12288 || K == 14336)) {  // rows of the large model widths
+    if (K == 12288) return launch_calib_smem_t<6>(x, rows, (int)K, ldb, gamma, beta, eps, out, st);
+    return launch_calib_smem_t<7>(x, rows, (int)K, ldb, gamma, beta, eps, out, st);
+  }
   int pT = 0, pn = 0;
   if (rowpipe_shape(K, bf16, 4, &pT, &pn))
     return launch_rowpipe_calib(x, bf16, rows, K, ld, gamma, beta, eps, out, pT, pn, st);

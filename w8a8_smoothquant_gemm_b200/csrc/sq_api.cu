@@ -3,7 +3,9 @@
 // any CUDA call, so a bad argument returns its status with nothing enqueued (and without
 // touching the device at all).
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "sq_common.cuh"
 
@@ -48,6 +50,33 @@ constexpr int kMaxDevices = 64;
 int g_sms[kMaxDevices];
 std::once_flag g_once[kMaxDevices];
 }  // namespace
+
+// Occupancy queries for clusters take long enough to show up in short kernels' launch time;
+// the answer depends only on the kernel, the device and the launch shape, so it is kept.
+cudaError_t max_active_clusters(const void* kern, const cudaLaunchConfig_t* cfg, int* clusters) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, size_t, unsigned, unsigned>, int> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  unsigned cx = 1;
+  for (unsigned i = 0; i < cfg->numAttrs; ++i)
+    if (cfg->attrs[i].id == cudaLaunchAttributeClusterDimension) cx = cfg->attrs[i].val.clusterDim.x;
+  const auto key = std::make_tuple(dev, kern, cfg->dynamicSmemBytes, cfg->blockDim.x, cx);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) {
+      *clusters = it->second;
+      return cudaSuccess;
+    }
+  }
+  e = cudaOccupancyMaxActiveClusters(clusters, kern, cfg);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = *clusters;
+  return cudaSuccess;
+}
 
 int num_sms() {
   int dev = 0;

@@ -249,5 +249,7 @@ __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
 // Host-side launch helpers (internal to the library; no C ABI).
 namespace sqh {
 int num_sms();                    // SM count of the current device (cached per device)
+// cudaOccupancyMaxActiveClusters, cached per device, kernel and launch shape
+cudaError_t max_active_clusters(const void* kern, const cudaLaunchConfig_t* cfg, int* clusters);
 unsigned int* error_word_ptr();   // device address of the error word (current device)
 }  // namespace sqh

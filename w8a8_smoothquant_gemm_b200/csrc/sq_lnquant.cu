@@ -391,11 +391,13 @@ static cudaError_t launch_rows(const void* x, bool bf16, int64_t M, int64_t K, i
                                const float* beta_f, const float* s, float eps, int8_t* xq, float* sx,
                                const float* scale_in, int write_codes, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
-  // LayerNorm rows of 12288 and 14336 below 4096 tokens: the block-per-row group kernel with
-  // exactly 6 or 7 chunks per thread (two blocks per SM) beats the chunk-pair kernel (one block
-  // of 8 warps per SM at 254 registers): 23.2 against 27.2 us at 2048 x 12288
-  const bool ln_long_few = gamma_f && bf16 && (K == 12288 || K == 14336) && M < 4096;
-  if (!ln_long_few && rowpair_supported(K, bf16, false, M))  // chunk-pair rows of the model widths
+  // LayerNorm rows of 12288 and 14336 and plain rows of 12288 below 4096 tokens: the
+  // block-per-row group kernel with exactly 6 or 7 chunks per thread (two blocks per SM) beats
+  // the chunk-pair kernel (one block of 8 warps per SM at 254 registers): 23.2 against 27.2 us
+  // (LayerNorm) and 32.0 against 34.8 us (plain) at 2048 x 12288; plain rows of 14336 measured
+  // 38.1 against 35.5 and stay on the chunk-pair kernel
+  const bool long_few = bf16 && M < 4096 && (K == 12288 || (gamma_f && K == 14336));
+  if (!long_few && rowpair_supported(K, bf16, false, M))  // chunk-pair rows of the model widths
     return launch_rowpair_quant(x, M, K, ldx, gamma_f, beta_f, s, eps, xq, sx, scale_in, write_codes, false, st);
   if (!gamma_f && K > 16384)  // long plain rows: split into segments, two passes
     return launch_rowsplit<false>(x, bf16, M, K, ldx, s, xq, sx, scale_in, write_codes, st);

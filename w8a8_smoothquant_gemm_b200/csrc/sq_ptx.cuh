@@ -86,9 +86,18 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
 // Barrier over every thread of every CTA of the cluster, with release/acquire ordering of
-// shared-memory writes (all threads of each CTA must call it).
+// shared-memory writes (all threads of each CTA must call it).  The barrier instructions are
+// warp-aligned, so the warp reconverges first (one lane may come from a longer branch, as
+// thread 0 of the cluster fold after it let its copies land).
 __device__ __forceinline__ void cluster_sync() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
@@ -99,6 +108,18 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// Reads 4 floats (16-byte aligned) from the shared memory of CTA `rank` of this cluster.
+__device__ __forceinline__ float4 ld_dsmem_f32x4(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(remote)
+               : "memory");
   return v;
 }
 
