@@ -55,6 +55,7 @@ struct GemmParams {
   int group_a;               // raster (b_major = 0): this many A tiles share a sweep over B tiles
   int group_b;               // raster (b_major = 1): this many B tiles share a sweep over A tiles
   int b_major;
+  int keep;                  // CTA pairs: 1 = A tiles, 2 = B tiles loaded with an L2 evict-last hint, 0 = none
   int M, N;                  // output is y[M, N]
   const float* sx;
   const float* sw;
@@ -82,6 +83,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// The same with an L2 cache-policy hint (createpolicy): the operand that every wave reads
+// again is kept in L2 ahead of the one that streams through.
+__device__ __forceinline__ void tma_load_2d_pair_keep(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                      uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
       : "memory");
 }
 
@@ -421,6 +432,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       bool ok = true;
       uint32_t issued = 0;  // bit s: stage s has been loaded; its last load used parity bit s of `par`
       uint32_t par = 0;
+      uint64_t keep_policy = 0;
+      if (CG == 2 && p.keep) asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep_policy));
       Work w = work_begin(p, unit0, unit_step);
       int ta, tb, kb0, kb1, split;
       while (ok && next_piece(p, w, ta, tb, kb0, kb1, split)) {
@@ -440,8 +453,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           } else {
             if (leader) mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(CG * L::STAGE_BYTES));
             const uint32_t fb = map_shared(full_bar(stage), 0);
-            tma_load_2d_pair(sa, &map_a, fb, kb * BK, ta * MMA_M + (int)rank * BM);
-            tma_load_2d_pair(sa + L::A_BYTES, &map_b, fb, kb * BK, tb * BN + (int)rank * L::BN_CTA);
+            const int ya = ta * MMA_M + (int)rank * BM, yb = tb * BN + (int)rank * L::BN_CTA;
+            if (p.keep == 1) tma_load_2d_pair_keep(sa, &map_a, fb, kb * BK, ya, keep_policy);
+            else tma_load_2d_pair(sa, &map_a, fb, kb * BK, ya);
+            if (p.keep == 2) tma_load_2d_pair_keep(sa + L::A_BYTES, &map_b, fb, kb * BK, yb, keep_policy);
+            else tma_load_2d_pair(sa + L::A_BYTES, &map_b, fb, kb * BK, yb);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -887,20 +903,29 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   p.kb_per_split = pl.kb_per_split;
   p.splits = pl.splits;
   p.num_units = pl.tiles_a * pl.tiles_b * pl.splits;
-  // Keep the smaller operand resident in L2 (up to ~48 MB of it per group) and stream the
-  // larger one through once.
+  // Tile order: the smaller operand's tiles are the fast index within a group, so the tiles
+  // one wave runs at once (they step through K together) share each K-block of both operands
+  // through L2.  A smaller operand of at most 64 MB forms one group and stays in L2 for the
+  // whole sweep (its loads carry an evict-last hint on CTA pairs); the larger one streams
+  // through once.  A larger smaller operand is taken about sqrt(CTA pairs) tiles at a time
+  // (square waves read the fewest tiles per wave).  Measured DRAM reads at 2048 x 12288 x
+  // 49152 with groups sized for 48 MB of L2: 2.74 GB for 0.70 GB of operands.
   {
-    const int64_t tile_m = (int64_t)sqk::BM * pl.cg, tile_n = pl.bn;
     const int64_t a_bytes = (pl.swap ? N : M) * K, b_bytes = (pl.swap ? M : N) * K;
-    const int64_t budget = 48ll << 20;
+    const int64_t resident = 64ll << 20;
+    const int64_t pairs = num_sms() / pl.cg;  // tiles that run at once
+    int64_t side = 1;
+    while (side * side < pairs) ++side;
     if (a_bytes <= b_bytes) {
       p.b_major = 0;
-      p.group_a = (int)std::max<int64_t>(1, std::min<int64_t>(pl.tiles_a, budget / std::max<int64_t>(1, tile_m * K)));
+      p.group_a = (int)(a_bytes <= resident ? pl.tiles_a : std::min<int64_t>(pl.tiles_a, side));
       p.group_b = 1;
+      p.keep = (pl.cg == 2 && a_bytes <= resident) ? 1 : 0;
     } else {
       p.b_major = 1;
-      p.group_b = (int)std::max<int64_t>(1, std::min<int64_t>(pl.tiles_b, budget / std::max<int64_t>(1, tile_n * K)));
+      p.group_b = (int)(b_bytes <= resident ? pl.tiles_b : std::min<int64_t>(pl.tiles_b, side));
       p.group_a = 1;
+      p.keep = (pl.cg == 2 && b_bytes <= resident) ? 2 : 0;
     }
   }
   p.M = (int)M;
