@@ -181,7 +181,7 @@ def test_fold_full_size(K, N):
 # ----------------------------------------------------------------------------- LN + smooth + quant
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
 @pytest.mark.parametrize("M,K", [(1, 16), (5, 256), (9, 1040), (33, 2048), (64, 4096), (7, 8192), (3, 12288),
-                                 (17, 14336), (4, 16384), (3, 16400), (2, 49152)])
+                                 (17, 14336), (4, 16384), (3, 16400), (2, 49152), (37, 20000), (513, 24576)])
 @pytest.mark.parametrize("mode", ["ln", "plain"])
 def test_ln_smooth_quant(dt, M, K, mode):
     if dt == "f32" and K > 32768:
@@ -446,6 +446,21 @@ def test_large_layer_sampled_rows(M, K, N, ln, w_std):
     assert np.array_equal(g["xq"][rows], xq) and np.array_equal(g["sx"][rows], sx)
     ref = O.w8a8_gemm(xq, sx, wq, sw, "bf16")
     assert assert_bf16_close(g["y"][rows], ref) == 1.0
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_long_plain_rows_divisors_outside_the_fast_range(dt):
+    """Rows longer than 16384 in plain mode divide by s through a reciprocal; a segment with a
+    factor outside [2^-90, 2^90] takes the correctly rounded division instead."""
+    M, K = 9, 20480
+    c = sq_inputs.make_case(M, K, 8, 77, x_dtype=dt, w_dtype=dt)
+    s = np.exp(np.random.default_rng(5).uniform(-1, 3, K)).astype(np.float32)
+    s[5] = np.float32(2.0 ** -100)   # first segment: huge quotients in channel 5
+    s[4100] = np.float32(2.0 ** 95)  # second segment: tiny quotients in channel 4100
+    xq, sx = sq.sq_ln_smooth_quant(dev(c.x), s=dev(s))
+    r_xq, r_sx = O.ln_smooth_quant(c.x, s=s)
+    assert np.array_equal(host(sx), r_sx)
+    assert np.array_equal(host(xq), r_xq)
 
 
 # ----------------------------------------------------------------------------- per-tensor granularity

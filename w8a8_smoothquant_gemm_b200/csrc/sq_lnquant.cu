@@ -159,82 +159,171 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
 
 
 // ---------------------------------------------------------------------------- long plain rows
-// Plain mode (y = x / s) on rows too long to hold in a thread group's registers (K > 16384):
-// each row is split into 8192-element segments, one block per (row, segment).  Pass 1 folds
-// the segment's max |y| into the row's slot of sx (float bits, atomicMax; sx starts at 0);
-// pass 2 recomputes y and writes the codes with scale = RN(max / 127) (or the given
-// per-tensor scale, codes clamped); pass 3 turns the maxima in sx into scales.  y = RN(x / s)
-// is the correctly rounded division.  (Blocks that own a segment for many rows, with s and
-// RN(1/s) staged once in shared memory, measured 2.3x slower: too few loads in flight.)
-constexpr int SEG_CHUNKS = 1024;  // 8192 elements per block: 256 threads x 4 chunks of 8
+// Plain mode (y = x / s) on rows too long to hold in a thread group's registers (K > 16384).
+// A block owns one segment of SEG_CH channels and strides over the rows (row p, p + P, ...).
+// Each thread keeps s and RN(1/s) of its SEG_CH / 2048 chunks in registers for all its rows,
+// so that y = RN(x / s) takes Markstein's three operations per element instead of a full
+// division (divisors outside the fast range fall back to the division, for the whole block).
+// Pass 1 folds each (row, segment) maximum of |y| into the row's slot of sx (float bits,
+// atomicMax; sx starts at 0); pass 2 recomputes y and writes the codes with scale =
+// RN(max / 127) (or the given per-tensor scale, codes clamped); pass 3 turns the maxima in sx
+// into scales.  Two rows per step, the next two rows' loads in flight behind them.
+// (One block per (row, segment) with a division per element: 153 us at 2048 x 49152.)
+constexpr int SEG_CH = 4096;                   // channels per segment
+constexpr int SEG_CPT = SEG_CH / 8 / 256;      // chunks per thread
+constexpr int SEG_CHUNKS = SEG_CH / 8;
 
 template <bool BF16>
-__device__ __forceinline__ void seg_load8(const char* row, int64_t c, float f[8]) {
+__device__ __forceinline__ void seg_load_raw(const char* row, int64_t c, uint4* v) {
   if (BF16) {
-    unpack8_bf16(ldg_stream16(row + c * 16), f);
+    v[0] = ldg_stream16(row + c * 16);
   } else {
-    const uint4 a = ldg_stream16(row + c * 32), b = ldg_stream16(row + c * 32 + 16);
-    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y); f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
-    f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y); f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+    v[0] = ldg_stream16(row + c * 32);
+    v[1] = ldg_stream16(row + c * 32 + 16);
   }
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(256)
-rowsplit_max_kernel(const char* __restrict__ x, int64_t K, int64_t ld_bytes, int64_t nseg,
-                    const float* __restrict__ s, float* __restrict__ rowmax) {
-  __shared__ float red[8];
-  const int64_t m = (int64_t)blockIdx.x / nseg, seg = (int64_t)blockIdx.x % nseg;
-  const int64_t nchunks = K / 8;
-  const char* row = x + m * ld_bytes;
-  float am = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t c = seg * SEG_CHUNKS + i * 256 + threadIdx.x;
-    if (c < nchunks) {
-      float f[8], y[8];
-      seg_load8<BF16>(row, c, f);
-      div_chunk(f, s, (int)c, y);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(y[e]));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float v = red[0];
-    for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w]);
-    atomic_max_nonneg(rowmax + m, v);
+__device__ __forceinline__ void seg_unpack(const uint4* v, float f[8]) {
+  if (BF16) {
+    unpack8_bf16(v[0], f);
+  } else {
+    f[0] = __uint_as_float(v[0].x); f[1] = __uint_as_float(v[0].y);
+    f[2] = __uint_as_float(v[0].z); f[3] = __uint_as_float(v[0].w);
+    f[4] = __uint_as_float(v[1].x); f[5] = __uint_as_float(v[1].y);
+    f[6] = __uint_as_float(v[1].z); f[7] = __uint_as_float(v[1].w);
   }
 }
 
-template <bool BF16, bool F8>
-__global__ void __launch_bounds__(256)
-rowsplit_codes_kernel(const char* __restrict__ x, int64_t K, int64_t ld_bytes, int64_t nseg,
-                      const float* __restrict__ s, const float* __restrict__ rowmax,
-                      const float* __restrict__ scale_in, int8_t* __restrict__ xq) {
-  const int64_t m = (int64_t)blockIdx.x / nseg, seg = (int64_t)blockIdx.x % nseg;
-  const int64_t nchunks = K / 8;
-  const char* row = x + m * ld_bytes;
-  const float scale = scale_in ? __ldg(scale_in) : __fdiv_rn(__ldg(rowmax + m), F8 ? 448.0f : 127.0f);
-  const SharedDivisor d(scale);
-  const bool clamp = scale_in != nullptr;
+// Per-thread channel constants of a segment: chunks c = seg * SEG_CHUNKS + t + 256 i.
+struct SegConst {
+  float s[SEG_CPT][8], rc[SEG_CPT][8];
+  bool ok[SEG_CPT];
+};
+
+__device__ __forceinline__ bool seg_const(SegConst& sc, const float* __restrict__ s, int64_t seg, int64_t nchunks) {
+  bool slow = false;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t c = seg * SEG_CHUNKS + i * 256 + threadIdx.x;
-    if (c < nchunks) {
-      float f[8], y[8];
-      seg_load8<BF16>(row, c, f);
-      div_chunk(f, s, (int)c, y);
-      uint2 w;
-      if (F8) w = d.fast ? pack8_e4m3<true>(y, d) : pack8_e4m3<false>(y, d);
-      else if (d.fast && !clamp) w = pack8_codes<true>(y, d);
-      else if (d.fast) w = pack8_codes<true, true>(y, d);
-      else w = pack8_codes<false, true>(y, d);
-      *reinterpret_cast<uint2*>(xq + m * K + c * 8) = w;
+  for (int i = 0; i < SEG_CPT; ++i) {
+    const int64_t c = seg * SEG_CHUNKS + threadIdx.x + 256 * i;
+    sc.ok[i] = c < nchunks;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float a = sc.ok[i] ? __ldg(s + c * 8 + e) : 1.0f;
+      const bool fast = fabsf(a) >= 0x1p-90f && fabsf(a) <= 0x1p+90f;
+      slow |= !fast;
+      sc.s[i][e] = a;
+      sc.rc[i][e] = fast ? __frcp_rn(a) : 0.0f;
     }
+  }
+  return slow;
+}
+
+// y = RN(x / s) for chunk i of the thread (FAST: Markstein on packed pairs).  SIGNED: the E4M3
+// codes tell -0 from +0, and RN(-0 / s) = -0, which Markstein's correction turns into +0.
+template <bool FAST, bool SIGNED>
+__device__ __forceinline__ void seg_div(const SegConst& sc, int i, const float f[8], float y[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    if (FAST) {
+      const float2 q = markstein2(make_float2(f[e], f[e + 1]), make_float2(sc.rc[i][e], sc.rc[i][e + 1]),
+                                  make_float2(-sc.s[i][e], -sc.s[i][e + 1]));
+      y[e] = SIGNED ? with_sign_of(q.x, f[e]) : q.x;
+      y[e + 1] = SIGNED ? with_sign_of(q.y, f[e + 1]) : q.y;
+    } else {
+      y[e] = __fdiv_rn(f[e], sc.s[i][e]);
+      y[e + 1] = __fdiv_rn(f[e + 1], sc.s[i][e + 1]);
+    }
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void seg_load_rows(const char* x, int64_t ld_bytes, int64_t r, int64_t M, int64_t seg,
+                                              const SegConst& sc, uint4 (&v)[2][SEG_CPT][BF16 ? 1 : 2]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int i = 0; i < SEG_CPT; ++i)
+      if (r + h < M && sc.ok[i])
+        seg_load_raw<BF16>(x + (r + h) * ld_bytes, seg * SEG_CHUNKS + threadIdx.x + 256 * i, v[h][i]);
+}
+
+// PASS 0: row maxima into rowmax; PASS 1: codes.  Block b: segment b % nseg, rows b / nseg,
+// b / nseg + P, ... in pairs (P = gridDim.x / nseg).
+template <bool BF16, int PASS, bool F8>
+__global__ void __launch_bounds__(256)
+rowsplit_kernel(const char* __restrict__ x, int64_t M, int64_t K, int64_t ld_bytes, int64_t nseg,
+                const float* __restrict__ s, float* __restrict__ rowmax, const float* __restrict__ scale_in,
+                int8_t* __restrict__ xq) {
+  constexpr int V = BF16 ? 1 : 2;
+  __shared__ float red[2][2][8];  // [step parity][row of the pair][warp]
+  const int64_t seg = blockIdx.x % nseg, p = blockIdx.x / nseg, P = gridDim.x / nseg;
+  const int64_t nchunks = K / 8;
+  SegConst sc;
+  const bool fast = !__syncthreads_or(seg_const(sc, s, seg, nchunks));
+  uint4 v[2][SEG_CPT][V], nv[2][SEG_CPT][V];
+  int64_t r = 2 * p;
+  if (r < M) seg_load_rows<BF16>(x, ld_bytes, r, M, seg, sc, v);
+  for (int step = 0; r < M; r += 2 * P, ++step) {
+    const int64_t rn = r + 2 * P;
+    if (rn < M) seg_load_rows<BF16>(x, ld_bytes, rn, M, seg, sc, nv);
+    if constexpr (PASS == 0) {
+      float am[2] = {0.0f, 0.0f};
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < SEG_CPT; ++i)
+          if (r + h < M && sc.ok[i]) {
+            float f[8], y[8];
+            seg_unpack<BF16>(v[h][i], f);
+            if (fast) seg_div<true, false>(sc, i, f, y);
+            else seg_div<false, false>(sc, i, f, y);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) am[h] = fmaxf(am[h], fabsf(y[e]));
+          }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) am[h] = fmaxf(am[h], __shfl_xor_sync(0xffffffffu, am[h], o));
+        if ((threadIdx.x & 31) == 0) red[step & 1][h][threadIdx.x >> 5] = am[h];
+      }
+      __syncthreads();  // red[step & 1] is rewritten two steps later, after the next barrier
+      if (threadIdx.x < 2 && r + threadIdx.x < M) {
+        float m = red[step & 1][threadIdx.x][0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, red[step & 1][threadIdx.x][w]);
+        atomic_max_nonneg(rowmax + r + threadIdx.x, m);
+      }
+    } else {
+      const bool clamp = scale_in != nullptr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (r + h >= M) continue;
+        const float scale = clamp ? __ldg(scale_in) : __fdiv_rn(__ldg(rowmax + r + h), F8 ? 448.0f : 127.0f);
+        const SharedDivisor d(scale);
+        int8_t* qrow = xq + (r + h) * K;
+#pragma unroll
+        for (int i = 0; i < SEG_CPT; ++i) {
+          if (!sc.ok[i]) continue;
+          float f[8], y[8];
+          seg_unpack<BF16>(v[h][i], f);
+          if (fast) seg_div<true, F8>(sc, i, f, y);
+          else seg_div<false, F8>(sc, i, f, y);
+          uint2 w;
+          if (F8) w = d.fast ? pack8_e4m3<true>(y, d) : pack8_e4m3<false>(y, d);
+          else if (d.fast && !clamp) w = pack8_codes<true>(y, d);
+          else if (d.fast) w = pack8_codes<true, true>(y, d);
+          else w = pack8_codes<false, true>(y, d);
+          *reinterpret_cast<uint2*>(qrow + (seg * SEG_CHUNKS + threadIdx.x + 256 * i) * 8) = w;
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < SEG_CPT; ++i)
+#pragma unroll
+        for (int u = 0; u < V; ++u) v[h][i][u] = nv[h][i][u];
   }
 }
 
@@ -353,31 +442,34 @@ cudaError_t launch_rowpair_quant(const void* x, int64_t M, int64_t K, int64_t ld
                                  const float* scale_in, int write_codes, bool f8, cudaStream_t st);
 
 
-// Plain-mode rows longer than the register-resident kernels hold (see rowsplit_*).  F8: E4M3
-// codes, scale = max / 448.
+// Plain-mode rows longer than the register-resident kernels hold (see rowsplit_kernel).  F8:
+// E4M3 codes, scale = max / 448.
 template <bool F8>
 static cudaError_t launch_rowsplit(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, const float* s,
                                    int8_t* xq, float* sx, const float* scale_in, int write_codes, cudaStream_t st) {
   const int64_t ldb = ldx * (bf16 ? 2 : 4);
   const int64_t nseg = (K / 8 + sqk::SEG_CHUNKS - 1) / sqk::SEG_CHUNKS;
-  const int64_t blocks = M * nseg;
+  // one wave: the row pairs of a segment spread over as many blocks as are resident at once
+  int per_sm = 1;
+  cudaError_t e = bf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sqk::rowsplit_kernel<true, 0, F8>, 256, 0)
+                       : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sqk::rowsplit_kernel<false, 0, F8>, 256, 0);
+  if (e != cudaSuccess) return e;
+  const int64_t pairs = (M + 1) / 2;
+  const int64_t per_seg = std::max<int64_t>(1, std::min<int64_t>(pairs, (int64_t)num_sms() * std::max(per_sm, 1) / nseg));
+  const int64_t blocks = nseg * per_seg;
   if (blocks > INT32_MAX) return cudaErrorInvalidValue;
-  cudaError_t e;
+  const char* xb = (const char*)x;
   if (!scale_in) {  // per-token maxima into sx
     e = cudaMemsetAsync(sx, 0, sizeof(float) * (size_t)M, st);
     if (e != cudaSuccess) return e;
-    if (bf16) sqk::rowsplit_max_kernel<true><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx);
-    else sqk::rowsplit_max_kernel<false><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx);
+    if (bf16) sqk::rowsplit_kernel<true, 0, F8><<<(unsigned)blocks, 256, 0, st>>>(xb, M, K, ldb, nseg, s, sx, scale_in, xq);
+    else sqk::rowsplit_kernel<false, 0, F8><<<(unsigned)blocks, 256, 0, st>>>(xb, M, K, ldb, nseg, s, sx, scale_in, xq);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (write_codes) {
-    if (bf16)
-      sqk::rowsplit_codes_kernel<true, F8><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx,
-                                                                            scale_in, xq);
-    else
-      sqk::rowsplit_codes_kernel<false, F8><<<(unsigned)blocks, 256, 0, st>>>((const char*)x, K, ldb, nseg, s, sx,
-                                                                             scale_in, xq);
+    if (bf16) sqk::rowsplit_kernel<true, 1, F8><<<(unsigned)blocks, 256, 0, st>>>(xb, M, K, ldb, nseg, s, sx, scale_in, xq);
+    else sqk::rowsplit_kernel<false, 1, F8><<<(unsigned)blocks, 256, 0, st>>>(xb, M, K, ldb, nseg, s, sx, scale_in, xq);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
