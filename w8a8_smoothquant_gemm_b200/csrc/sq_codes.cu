@@ -22,6 +22,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(256)
 quant_codes_kernel(const char* __restrict__ x, int64_t K, int64_t ld_bytes, const float* __restrict__ rowmax,
                    int8_t* __restrict__ xq, float* __restrict__ sx) {
+  allow_dependent_launch();
   const int64_t m = blockIdx.y;
   const float scale = __fdiv_rn(__ldg(rowmax + m), 127.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) sx[m] = scale;

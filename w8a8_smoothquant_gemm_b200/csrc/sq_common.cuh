@@ -239,6 +239,16 @@ __device__ __forceinline__ uint4 ldg_stream16(const void* p) {
   return v;
 }
 
+// Lets the next kernel on the stream start its set-up, if it was launched as a programmatic
+// dependent (the GEMM is: it allocates TMEM, initialises its barriers and asks L2 for its first
+// weight tiles, and reads nothing that this kernel writes before its griddepcontrol.wait, which
+// returns once this grid has completed and its writes are visible).  The quantisers call it
+// first thing, so that in decode the GEMM's weight stream starts while the activations are
+// quantised.  No effect when the next kernel is an ordinary launch.
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Max of non-negative floats through their bit patterns (monotone for x >= +0).
 __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
   atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));

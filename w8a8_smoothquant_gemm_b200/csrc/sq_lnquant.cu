@@ -26,6 +26,7 @@ ln_smooth_quant_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_
                        const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
                        const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
                        const float* __restrict__ scale_in, int write_codes) {
+  allow_dependent_launch();
   __shared__ float red[3 * (ROW_WARPS + 1)];
   const int nchunks = K / 8;
   RowChunks<BF16, MAXC> cur;
@@ -93,6 +94,7 @@ ln_quant_group_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_b
                       const float* __restrict__ gamma_f, const float* __restrict__ beta_f,
                       const float* __restrict__ s, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
                       const float* __restrict__ scale_in, int write_codes, int use_table) {
+  allow_dependent_launch();
   constexpr int G = 256 / T;
   __shared__ float red[G][24];  // per group: mean partials, variance partials, max
   extern __shared__ float rs[];  // plain mode: RN(1 / s_j), or 0 where s_j is outside the fast range
@@ -255,6 +257,7 @@ __global__ void __launch_bounds__(256)
 rowsplit_kernel(const char* __restrict__ x, int64_t M, int64_t K, int64_t ld_bytes, int64_t nseg,
                 const float* __restrict__ s, float* __restrict__ rowmax, const float* __restrict__ scale_in,
                 int8_t* __restrict__ xq) {
+  allow_dependent_launch();
   constexpr int V = BF16 ? 1 : 2;
   __shared__ float red[2][2][8];  // [step parity][row of the pair][warp]
   const int64_t seg = blockIdx.x % nseg, p = blockIdx.x / nseg, P = gridDim.x / nseg;
@@ -330,12 +333,14 @@ rowsplit_kernel(const char* __restrict__ x, int64_t M, int64_t K, int64_t ld_byt
 // sx[m] = RN(max_m / 127) (F8: / 448), or the given per-tensor scale.
 template <bool F8>
 __global__ void rowsplit_scales_kernel(float* __restrict__ sx, int64_t M, const float* __restrict__ scale_in) {
+  allow_dependent_launch();
   const int64_t m = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (m < M) sx[m] = scale_in ? __ldg(scale_in) : __fdiv_rn(sx[m], F8 ? 448.0f : 127.0f);
 }
 
 // out[0] = max of v[0 .. n) (non-negative floats), one block.
 __global__ void __launch_bounds__(1024) max_of_vector_kernel(const float* __restrict__ v, int64_t n, float* out) {
+  allow_dependent_launch();
   __shared__ float red[32];
   float m = 0.0f;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, v[i]);

@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(32 * W, 1)
 rowpair_kernel(const char* __restrict__ x, int64_t M, int64_t ld_bytes, const float* __restrict__ vec_a,
                const float* __restrict__ vec_b, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
                float* __restrict__ out, const float* __restrict__ scale_in, int write_codes) {
+  allow_dependent_launch();
   constexpr int NT = 32 * W;
   constexpr int G = NT / T;
   constexpr int P = 256 / T;

@@ -26,6 +26,7 @@ __global__ void __launch_bounds__(256)
 rowpipe_kernel(const char* __restrict__ x, int64_t M, int K, int64_t ld_bytes, const float* __restrict__ vec_a,
                const float* __restrict__ vec_b, float eps, int8_t* __restrict__ xq, float* __restrict__ sx,
                float* __restrict__ out, const float* __restrict__ scale_in, int write_codes, unsigned int* err) {
+  allow_dependent_launch();
   constexpr int G = 256 / T;
   constexpr int ELT = BF16 ? 2 : 4;
   constexpr bool LN = MODE != ROW_PLAIN_QUANT;
