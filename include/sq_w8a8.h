@@ -171,7 +171,10 @@ sq_status sq_ln_smooth_quant_per_tensor(const void* x, sq_dtype dt, int64_t M, i
  *   and every call leaves all of it zero-filled again, so one
  *   workspace serves any number of calls and shapes (and the FP8 GEMM) without clearing.  (A
  *   call whose kernel stopped on a bounded wait -- sq_device_error() != 0 -- may leave it
- *   dirty: zero it again.)  Calls that share a workspace must be ordered on one stream. */
+ *   dirty: zero it again.)  Calls that share a workspace must be ordered on one stream.
+ *   For M > 128 with many output tiles the workspace is optional: it lets the last, short
+ *   wave of tiles be split along K over all SMs (summed by a second kernel); with a smaller
+ *   or NULL workspace those tiles run whole, with the same result. */
 sq_status sq_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                        int64_t M, int64_t N, int64_t K, void* y, sq_dtype ydt, int64_t ldy,
                        void* workspace, size_t ws_bytes, void* stream);

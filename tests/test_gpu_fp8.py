@@ -130,6 +130,24 @@ def test_gemm_fp8_accumulator(M, N, K):
     assert np.all(err <= _acc_bound(xq, wq)), float(np.max(err / np.maximum(_acc_bound(xq, wq), 1e-300)))
 
 
+def test_gemm_fp8_split_tail_sampled_rows():
+    """CTA-pair tiles in a full wave plus two tiles split along K over the idle pairs (300 x
+    9572 x 16400): the pieces' fp32 partials are summed in split order; sampled rows, every
+    column, within the bound."""
+    M, N, K = 300, 9572, 16400
+    rng = np.random.default_rng(41)
+    xq, wq = _finite_codes(rng, (M, K)), _finite_codes(rng, (N, K))
+    ones_m, ones_n = np.ones(M, np.float32), np.ones(N, np.float32)
+    ws = torch.zeros(sq.sq_w8a8_gemm_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+    got = host(sq.sq_w8a8_gemm_fp8(dev(xq), dev(ones_m), dev(wq), dev(ones_n), out_dtype=torch.float32,
+                                   workspace=ws))
+    assert not ws.any()
+    r = np.array([0, 1, 128, 255, 256, 299])
+    exact, _ = O.fp8_gemm(xq[r], ones_m[r], wq, ones_n, "f32")
+    err = np.abs(got[r].astype(np.float64) - exact)
+    assert np.all(err <= _acc_bound(xq[r], wq))
+
+
 def test_gemm_fp8_and_int8_share_a_workspace():
     """FP8 and INT8 GEMMs of split shapes take turns on one zero-filled workspace: every result
     holds (FP8 within its bound, and the same bits on a repeated call; INT8 exact) and the

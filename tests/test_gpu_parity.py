@@ -4,6 +4,8 @@ int8 codes and int32 accumulators; bf16 outputs within 1 bf16 ulp or 4e-3 relati
 kernels take the oracle's exact sequence of roundings, so they are in fact bit-identical,
 which the tests also record).  Small cases are compared in full; full-size workloads on
 sampled rows (every column of those rows)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -550,3 +552,49 @@ def test_next_smoothing_folded_into_previous_linear():
     assert np.array_equal(host(yA2), r_yA2)
     assert np.array_equal(host(xqB), r_xqB) and np.array_equal(host(sxB), r_sxB)
     assert np.array_equal(host(yB), r_yB)
+
+
+
+# A full wave of CTA-pair tiles plus a short last wave: 2 x 38 = 76 tiles on 74 pairs, long K,
+# so the last two tiles are split along K over the idle pairs and a second kernel sums the
+# pieces.  Ragged last row tile (300 rows), column tile (9572 columns) and last K piece.
+SPLIT_TAIL = (300, 9572, 16400)
+SPLIT_ROWS = np.array([0, 1, 127, 128, 255, 256, 299])
+
+
+def test_split_tail_gemm_sampled_rows():
+    M, N, K = SPLIT_TAIL
+    assert sq.sq_w8a8_gemm_workspace_size(M, N, K) > 0
+    rng = np.random.default_rng(31)
+    xq, wq = random_codes(rng, M, K, extreme_row=0), random_codes(rng, N, K)
+    sx = rng.uniform(1e-3, 0.5, M).astype(np.float32)
+    sw = rng.uniform(1e-5, 1e-2, N).astype(np.float32)
+    dx, dw, dsx, dsw = dev(xq), dev(wq), dev(sx), dev(sw)
+    ws = torch.zeros(sq.sq_w8a8_gemm_workspace_size(M, N, K), dtype=torch.uint8, device=DEV)
+    acc = host(sq.sq_w8a8_gemm(dx, None, dw, None, out_dtype=torch.int32, workspace=ws))
+    assert not ws.any()
+    r = SPLIT_ROWS
+    assert np.array_equal(acc[r], O.w8a8_gemm(xq[r], None, wq, None, "i32"))
+    y, rmax = sq.sq_w8a8_gemm_rowmax(dx, dsx, dw, dsw, workspace=ws)
+    assert not ws.any()
+    ref = O.w8a8_gemm(xq[r], sx[r], wq, sw, "bf16")
+    assert np.array_equal(host(y)[r], ref)
+    assert np.array_equal(host(rmax)[r], O.calib_absmax(ref, 1))
+
+
+def test_split_tail_is_optional():
+    """The split tail needs a workspace; given none, the call runs the last tiles whole, with
+    the same exact result."""
+    M, N, K = SPLIT_TAIL
+    rng = np.random.default_rng(17)
+    xq, wq = random_codes(rng, M, K, extreme_row=0), random_codes(rng, N, K)
+    dx, dw = dev(xq), dev(wq)
+    with_ws = host(sq.sq_w8a8_gemm(dx, None, dw, None, out_dtype=torch.int32))
+    without = torch.empty(M, N, dtype=torch.int32, device=DEV)
+    f = sq.lib().sq_w8a8_gemm
+    assert f(ctypes.c_void_p(dx.data_ptr()), None, ctypes.c_void_p(dw.data_ptr()), None, M, N, K,
+             ctypes.c_void_p(without.data_ptr()), sq.SQ_I32, N, None, 0,
+             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    r = SPLIT_ROWS
+    assert np.array_equal(with_ws, host(without))
+    assert np.array_equal(with_ws[r], O.w8a8_gemm(xq[r], None, wq, None, "i32"))

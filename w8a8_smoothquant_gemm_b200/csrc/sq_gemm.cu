@@ -63,7 +63,11 @@ struct GemmParams {
   int64_t ldy;
   int ydt;                   // SQ_BF16, SQ_F32 or SQ_I32
   int vec_store;             // y and every output row start on a 16-byte boundary
-  int32_t* ws;               // [splits][M][N] int32 partials when splits > 1
+  int32_t* ws;               // [splits][M][N] int32 partials when splits > 1; with hy, the tail tiles' partials
+  // split tail (CTA pairs): the first hy_dp tiles (whole waves) go whole; each of the hy_tail
+  // remaining tiles is cut into hy_splits runs of hy_kbps K blocks, one unit each, whose
+  // partial tiles go to ws as [hy_splits][hy_tail][256 rows][BN] int32 (FP8: fp32 bits)
+  int hy, hy_dp, hy_tail, hy_splits, hy_kbps;
   // stream-K (swap layout only): the first sk_dp_tiles tiles go whole to the CTAs in full waves
   // (tile u to CTA u mod G); of the rest, CTA c of G = sk_ctas takes iterations
   // [c I / G, (c+1) I / G) of their I = (tiles_a - sk_dp_tiles) * num_kb (tile, K block)
@@ -255,9 +259,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // concurrently.  Tiles are rastered so that one operand stays resident in L2 while the
 // other streams through once: a group of group_a A tiles sweeps over all B tiles (A tile
 // index fastest), or, with b_major, a group of group_b B tiles sweeps over all A tiles.
-__device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta, int& tb, int& split) {
-  split = u % p.splits;
-  const int tile = u / p.splits;
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& ta, int& tb) {
   if (!p.b_major) {
     const int group_size = p.group_a * p.tiles_b;
     const int group = tile / group_size;
@@ -277,18 +279,25 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta,
   }
 }
 
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& ta, int& tb, int& split) {
+  split = u % p.splits;
+  tile_coords(p, u / p.splits, ta, tb);
+}
+
 // The sequence of pieces (tile, K-block range) one CTA works on.  Data-parallel: units
 // unit0, unit0 + step, ... (decode_unit).  Stream-K: the CTA's iteration range, cut at tile
 // boundaries (the first and last piece may be partial tiles).
 struct Work {
   int64_t it, end;  // stream-K cursor
   int u, step;      // data-parallel cursor
+  int tail;         // split tail: index of the current piece's tile among the tail tiles, or -1
 };
 
 __device__ __forceinline__ Work work_begin(const GemmParams& p, int unit0, int unit_step) {
   Work w;
   w.u = unit0;
   w.step = unit_step;
+  w.tail = -1;
   w.it = (int64_t)unit0 * p.sk_iters / p.sk_ctas;
   w.end = (int64_t)(unit0 + 1) * p.sk_iters / p.sk_ctas;
   return w;
@@ -315,6 +324,25 @@ __device__ __forceinline__ bool next_piece(const GemmParams& p, Work& w, int& ta
     return true;
   }
   if (w.u >= p.num_units) return false;
+  if (p.hy) {
+    const int u = w.u;
+    w.u += w.step;
+    if (u < p.hy_dp) {  // a whole tile of the full waves
+      tile_coords(p, u, ta, tb);
+      split = 0;
+      kb0 = 0;
+      kb1 = p.num_kb;
+      w.tail = -1;
+      return true;
+    }
+    const int v = u - p.hy_dp;
+    w.tail = v / p.hy_splits;
+    split = v % p.hy_splits;
+    tile_coords(p, p.hy_dp + w.tail, ta, tb);
+    kb0 = split * p.hy_kbps;
+    kb1 = min(p.num_kb, kb0 + p.hy_kbps);
+    return true;
+  }
   decode_unit(p, w.u, ta, tb, split);
   kb0 = split * p.kb_per_split;
   kb1 = min(p.num_kb, kb0 + p.kb_per_split);
@@ -560,6 +588,27 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         if (lane == 0) mbar_arrive(tempty_bar(acc));
         continue;
       }
+      if (!SWAP && p.hy && w.tail >= 0) {
+        // ---- a piece of a split tail tile: the raw partial (int32, or fp32 bits) into its slot;
+        // the reduction kernel that follows this grid sums the pieces in split order
+        int32_t* dst = p.ws + (((int64_t)split * p.hy_tail + w.tail) * MMA_M + (int64_t)rank * BM + row) * BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += CH) {
+          uint32_t r[CH];
+          tmem_ld<CH>(taddr + (uint32_t)c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < CH; i += 4)
+            *reinterpret_cast<uint4*>(dst + c0 + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 1) mbar_arrive(tempty_bar(acc));
+          else mbar_arrive_cluster(map_shared(tempty_bar(acc), 0));
+        }
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += CH) {
         uint32_t r[CH];
@@ -693,6 +742,54 @@ splitk_reduce_kernel(int32_t* __restrict__ ws, int splits, int64_t M, int64_t N,
   }
 }
 
+// Finishes the split tail tiles of a CTA-pair GEMM: y = epilogue(sum of the pieces in split
+// order: int32 exact, FP8 fp32 in that fixed order), the row maxima for rowmax, and the pieces
+// back to zero.  Thread: four consecutive columns of one row of one tail tile.
+template <bool F8>
+__global__ void __launch_bounds__(256)
+hy_reduce_kernel(const GemmParams p, int bn) {
+  allow_dependent_launch();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the GEMM grid has completed
+  const int per_tile = 256 * bn / 4;                  // 4-column groups of one tail tile
+  const int64_t total = (int64_t)p.hy_tail * per_tile;
+  const int64_t slab = (int64_t)p.hy_tail * 256 * bn;  // one split's pieces
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total; g += (int64_t)gridDim.x * blockDim.x) {
+    const int t = (int)(g / per_tile), e = (int)(g % per_tile);
+    const int r = e / (bn / 4), c = (e % (bn / 4)) * 4;
+    int ta, tb;
+    tile_coords(p, p.hy_dp + t, ta, tb);
+    const int64_t m = (int64_t)ta * 256 + r, n0 = (int64_t)tb * bn + c;
+    int32_t* src = p.ws + ((int64_t)t * 256 + r) * bn + c;
+    uint32_t acc[4];
+    if (F8) {
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < p.hy_splits; ++s) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + s * slab);
+        a[0] = __fadd_rn(a[0], __uint_as_float(v.x)); a[1] = __fadd_rn(a[1], __uint_as_float(v.y));
+        a[2] = __fadd_rn(a[2], __uint_as_float(v.z)); a[3] = __fadd_rn(a[3], __uint_as_float(v.w));
+        *reinterpret_cast<uint4*>(src + s * slab) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      for (int i = 0; i < 4; ++i) acc[i] = __float_as_uint(a[i]);
+    } else {
+      int32_t a[4] = {0, 0, 0, 0};
+      for (int s = 0; s < p.hy_splits; ++s) {
+        const int4 v = *reinterpret_cast<const int4*>(src + s * slab);
+        a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+        *reinterpret_cast<int4*>(src + s * slab) = make_int4(0, 0, 0, 0);
+      }
+      for (int i = 0; i < 4; ++i) acc[i] = (uint32_t)a[i];
+    }
+    if (m >= p.M) continue;
+    const float sxm = p.ydt == SQ_I32 ? 0.0f : __ldg(p.sx + m);
+    float rmax = 0.0f;
+    for (int i = 0; i < 4; ++i) {
+      const int64_t n = n0 + i;
+      if (n < p.N) rmax = fmaxf(rmax, store_out<F8>(p, m, n, acc[i], sxm, p.ydt == SQ_I32 ? 0.0f : __ldg(p.sw + n)));
+    }
+    if (p.rowmax) atomic_max_nonneg(p.rowmax + m, rmax);
+  }
+}
+
 // Finishes the tiles of a stream-K GEMM that several CTAs shared: y = epilogue(sum of the
 // partial tiles), and the workspace back to zero.  INT8: the int32 tile sum; FP8: the
 // contributors' slots added in K order.  Block b covers 1024 elements of split tile b / (BN / 8)
@@ -796,10 +893,14 @@ struct GemmPlan {
   bool sk;          // stream-K split of the swap layout
   int sk_ctas, sk_dp_tiles;
   int64_t sk_iters;
-  size_t ws_bytes;  // 0, or the split-K partials / stream-K tile sums (zero at rest)
+  bool hy;          // split tail of the CTA-pair layout
+  int hy_dp, hy_tail, hy_splits, hy_kbps;
+  size_t ws_bytes;  // 0, or the split-K partials / stream-K tile sums / split-tail pieces (zero at rest)
 };
 
-static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
+// split_tail = false: the plan without the split tail (which is the only part of a CTA-pair
+// plan with many tiles that needs a workspace).
+static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, bool split_tail = true) {
   GemmPlan pl{};
   const int sms = num_sms();
   pl.swap = M <= 128;
@@ -846,10 +947,30 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
   pl.kb_per_split = (pl.num_kb + splits - 1) / splits;
   pl.splits = (pl.num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
   pl.ws_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(int32_t) : 0;
+  // Split tail: when the last wave holds at most half as many tiles as there are CTA pairs,
+  // its tiles are cut along K so that all pairs share it; the full waves keep whole tiles.
+  // Only for long K (pieces of at least 64 K blocks): 2048 x 12288 x 49152 (5 waves of 74
+  // tiles and 14) measured 734 against 780 us, while pieces of 16-20 K blocks cost more than
+  // the short wave they save (2048 x 12288 x 12288: 202 against 200 us; 8192 x 6144 x 4096:
+  // 160-179 against 138-142 us): a piece writes a whole 256 x 256 partial tile.
+  if (split_tail && tiles >= slots) {
+    const int64_t tail = tiles % slots;
+    const int64_t hs = tail ? std::min<int64_t>(slots / tail, pl.num_kb / 64) : 0;
+    if (hs >= 2) {
+      pl.hy = true;
+      pl.hy_dp = (int)(tiles - tail);
+      pl.hy_tail = (int)tail;
+      pl.hy_kbps = (int)((pl.num_kb + hs - 1) / hs);
+      pl.hy_splits = (pl.num_kb + pl.hy_kbps - 1) / pl.hy_kbps;
+      pl.ws_bytes = (size_t)pl.hy_splits * (size_t)tail * tile_m * (size_t)pl.bn * sizeof(int32_t);
+    }
+  }
   return pl;
 }
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K) { return plan_gemm(M, N, K).ws_bytes; }
+// The smallest workspace a launch of this shape can run with (no split tail).
+size_t gemm_workspace_size_min(int64_t M, int64_t N, int64_t K) { return plan_gemm(M, N, K, false).ws_bytes; }
 
 template <int BN, int STAGES, bool SWAP, int CG, bool F8>
 static cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const sqk::GemmParams& p,
@@ -882,7 +1003,9 @@ template <bool F8>
 static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* wq, const float* sw, int64_t M,
                                    int64_t N, int64_t K, void* y, int ydt, int64_t ldy, void* ws, size_t ws_bytes,
                                    float* rowmax, cudaStream_t st, bool* ws_too_small) {
-  const GemmPlan pl = plan_gemm(M, N, K);
+  GemmPlan pl = plan_gemm(M, N, K);
+  // a workspace too small for the split tail: the plan without it (which needs none)
+  if (pl.hy && (ws == nullptr || ws_bytes < pl.ws_bytes)) pl = plan_gemm(M, N, K, false);
   *ws_too_small = pl.ws_bytes > 0 && (ws == nullptr || ws_bytes < pl.ws_bytes);
   if (*ws_too_small) return cudaSuccess;
   if (rowmax) {  // the epilogue takes a running max into it
@@ -902,7 +1025,12 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
   p.num_kb = pl.num_kb;
   p.kb_per_split = pl.kb_per_split;
   p.splits = pl.splits;
-  p.num_units = pl.tiles_a * pl.tiles_b * pl.splits;
+  p.num_units = pl.hy ? pl.hy_dp + pl.hy_tail * pl.hy_splits : pl.tiles_a * pl.tiles_b * pl.splits;
+  p.hy = pl.hy ? 1 : 0;
+  p.hy_dp = pl.hy_dp;
+  p.hy_tail = pl.hy_tail;
+  p.hy_splits = pl.hy ? pl.hy_splits : 1;
+  p.hy_kbps = pl.hy_kbps;
   // Tile order: the smaller operand's tiles are the fast index within a group, so the tiles
   // one wave runs at once (they step through K together) share each K-block of both operands
   // through L2.  A smaller operand of at most 64 MB forms one group and stays in L2 for the
@@ -970,6 +1098,20 @@ static cudaError_t launch_gemm_any(const void* xq, const float* sx, const void* 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, sqk::sk_reduce_kernel<F8>, p, pl.bn);
+  }
+  if (pl.hy) {
+    // the split tail's reduction, a programmatic dependent of the GEMM
+    const int64_t groups = (int64_t)pl.hy_tail * 256 * pl.bn / 4;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>((groups + 255) / 256, (int64_t)num_sms() * 8));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, sqk::hy_reduce_kernel<F8>, p, pl.bn);
   }
   if (pl.splits == 1) return e;
   const int64_t total = M * N;

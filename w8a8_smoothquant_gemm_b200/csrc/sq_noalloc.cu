@@ -22,6 +22,10 @@ sq_status check_gemm_args(const int8_t* xq, const float* sx, const int8_t* wq, c
                           int64_t K, const void* y, sq_dtype ydt, int64_t ldy, bool* empty);
 }
 
+namespace sqh {
+size_t gemm_workspace_size_min(int64_t M, int64_t N, int64_t K);
+}  // namespace sqh
+
 namespace {
 
 static __device__ __align__(256) unsigned char g_gemm_scratch[SQ_NOALLOC_SCRATCH_BYTES];
@@ -61,7 +65,9 @@ extern "C" sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* sx, con
   bool empty = false;
   const sq_status st = sqh::check_gemm_args(xq, sx, wq, sw, M, N, K, y, ydt, ldy, &empty);
   if (st != SQ_OK || empty) return st;
-  const size_t need = sq_w8a8_gemm_workspace_size(M, N, K);
+  // the smallest workspace a launch of this shape runs with (the split tail of large CTA-pair
+  // shapes is optional and not used here)
+  const size_t need = sqh::gemm_workspace_size_min(M, N, K);
   if (need == 0) return sq_w8a8_gemm(xq, sx, wq, sw, M, N, K, y, ydt, ldy, nullptr, 0, stream);
   if (need > (size_t)SQ_NOALLOC_SCRATCH_BYTES) return SQ_ERR_WORKSPACE;
   void* scratch = nullptr;
