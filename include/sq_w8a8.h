@@ -221,8 +221,10 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *   library holds until the process exits.  The caller still passes all inputs and
  *   outputs, with the same meaning, layout and checks as sq_w8a8_gemm.
  *   - The arguments are checked first, in the order sq_w8a8_gemm checks them; then a shape
- *     whose workspace (sq_w8a8_gemm_workspace_size) exceeds the scratch returns
- *     SQ_ERR_WORKSPACE with nothing launched.
+ *     whose required workspace exceeds the scratch returns SQ_ERR_WORKSPACE with nothing
+ *     launched.  The required workspace is sq_w8a8_gemm_workspace_size's, except for large
+ *     CTA-pair shapes, whose optional split tail (see sq_w8a8_gemm) this entry point does
+ *     not use: they run with no scratch at all.
  *   - The first call on a device looks up the scratch array's device address (set-up, once
  *     per device, with that device current); make that first call before any stream
  *     capture.  A failed look-up returns SQ_ERR_CUDA.
