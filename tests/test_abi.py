@@ -253,3 +253,27 @@ def test_fold_kernel_launches_routing():
     assert f(A16, BF16, 49152, 64, 64) == 3                # cluster block too tall
     assert f(A8, BF16, 49152, 64, 64) == 1                 # unaligned: strip kernel
     assert f(A16, F32, 4096, 28672, 28672) == 1            # fp32 weights: strip kernel
+
+
+def test_workspace_sizes_follow_the_launch_plan():
+    """Host-only launch planning (148 SMs when no device answers, as on a B200): the workspace
+    each GEMM shape asks for, derived by hand from the planning rules."""
+    ws = sq.sq_w8a8_gemm_workspace_size
+    # swap-AB decode, 32 weight tiles on 148 SMs: stream-K over all 148 CTAs; the larger of the
+    # tile sums (32 tiles) and two partial slots per CTA (296), of 128 x BN int32 (BN = 16)
+    assert ws(1, 4096, 4096) == 296 * 128 * 16 * 4
+    # 224 tiles: one full wave of whole tiles, then 76 tiles stream-K over 148 CTAs
+    assert ws(16, 28672, 4096) == 296 * 128 * 16 * 4
+    # BN = 64 for 33-64 tokens
+    assert ws(64, 4096, 14336) == 296 * 128 * 64 * 4
+    # CTA pairs, 36 tiles on 74 pairs: K split 2 ways, [2][M][N] int32
+    assert ws(1536, 1536, 4096) == 2 * 1536 * 1536 * 4
+    # CTA pairs, 384 tiles = 5 waves of 74 + 14, K = 384 blocks: the 14 tail tiles in 5 pieces
+    # of 77 blocks, [5][14][256][256] int32
+    assert ws(2048, 12288, 49152) == 5 * 14 * 256 * 256 * 4
+    # the same tiling with K = 96 blocks: pieces would be shorter than 64 blocks, no split tail
+    assert ws(2048, 12288, 12288) == 0
+    # 76 tiles = 74 + 2, K = 129 blocks: 2 pieces (65 + 64 blocks) per tail tile
+    assert ws(300, 9572, 16400) == 2 * 2 * 256 * 256 * 4
+    # 768 tiles = 10 waves + 28, K = 32 blocks: no split tail
+    assert ws(8192, 6144, 4096) == 0
