@@ -277,3 +277,15 @@ def test_workspace_sizes_follow_the_launch_plan():
     assert ws(300, 9572, 16400) == 2 * 2 * 256 * 256 * 4
     # 768 tiles = 10 waves + 28, K = 32 blocks: no split tail
     assert ws(8192, 6144, 4096) == 0
+
+
+def test_binding_has_no_fallback(monkeypatch):
+    """Without the library every call raises; host tensors are refused, not computed on the CPU."""
+    import torch
+    x = torch.zeros(2, 16)
+    with pytest.raises(ValueError):
+        sq.sq_ln_smooth_quant(x, s=torch.ones(16))
+    monkeypatch.setattr(sq, "_lib", None)
+    monkeypatch.setattr(sq, "LIB_PATH", os.path.join(ROOT, "w8a8_smoothquant_gemm_b200", "no_such_library.so"))
+    with pytest.raises(OSError):
+        sq.lib()
